@@ -1,0 +1,236 @@
+"""Python binding of libeffort, the B200 library for the Effort approximate matvec.
+
+Argument marshalling only: tensors are passed to the C ABI of
+``include/effort.h`` as raw device pointers with torch's current CUDA stream;
+every step of the computation runs in the library's CUDA kernels.  There is no
+fallback: if ``libeffort.so`` is missing or a call fails, an exception is
+raised.
+
+Method: Hacker News item 40067677, "Show HN: Speeding up LLM inference 2x times
+(possibly)" -- rows sorted by |w|, probes, cutoff = topK(v * probes, effort),
+multiply over the used leading part of every row.
+"""
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libeffort.so")
+
+F32, F16 = 0, 1
+STATUS = {0: "ok", 1: "invalid argument", 2: "CUDA error", 3: "out of memory",
+          4: "non-finite input", 5: "device-side inconsistency", 6: "unsupported size"}
+MAX_OUT_DIM = 32768
+MAX_IN_DIM = 40960
+
+_lib = None
+
+
+class EffortError(RuntimeError):
+    def __init__(self, status, what):
+        super().__init__(f"{what}: {STATUS.get(status, status)} (status {status})")
+        self.status = status
+
+
+class Layout(ctypes.Structure):
+    _fields_ = [("in_dim", ctypes.c_int64), ("out_dim", ctypes.c_int64),
+                ("n_kept", ctypes.c_int32), ("n_tiles", ctypes.c_int32), ("bucket_cap", ctypes.c_int32),
+                ("ck_step", ctypes.c_int32), ("n_ck", ctypes.c_int32), ("n_probes", ctypes.c_int32),
+                ("vals", ctypes.c_void_p), ("idx", ctypes.c_void_p), ("probes", ctypes.c_void_p),
+                ("ckmag", ctypes.c_void_p), ("cnt", ctypes.c_void_p), ("wdense", ctypes.c_void_p),
+                ("rec", ctypes.c_void_p), ("gcnt", ctypes.c_void_p), ("n_groups", ctypes.c_int32)]
+
+
+def lib():
+    """Load libeffort.so (built in-tree by dynamic_approximate_gemv_b200.build)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: run `python -m dynamic_approximate_gemv_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i64, i32, f32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float
+        sig = {
+            "effort_prepare": [vp, i64, i64, f32, vp, ctypes.POINTER(vp)],
+            "effort_gemv": [vp, vp, f32, vp, vp],
+            "effort_gemv_ex": [vp, vp, ctypes.c_int, f32, vp, vp, vp, vp, vp],
+            "effort_check": [vp],
+            "effort_workspace_create": [i64, i64, i32, ctypes.POINTER(vp)],
+            "effort_workspace_destroy": [vp],
+            "effort_gemv_batched": [vp, vp, vp, vp, i32, vp, ctypes.c_int, vp, vp, vp, vp, vp],
+            "effort_dense_gemv": [vp, vp, i64, i64, vp, ctypes.c_int, vp, vp],
+            "effort_get_info": [vp, ctypes.POINTER(i64), ctypes.POINTER(i64), ctypes.POINTER(f32),
+                                ctypes.POINTER(ctypes.c_size_t)],
+            "effort_get_layout": [vp, ctypes.POINTER(Layout)],
+            "effort_destroy": [vp],
+        }
+        for name, args in sig.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = ctypes.c_int
+        L.effort_status_string.argtypes = [ctypes.c_int]
+        L.effort_status_string.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def _check(status, what):
+    if status != 0:
+        raise EffortError(status, what)
+
+
+def _stream(device=None):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _vdtype(v):
+    if v.dtype == torch.float32:
+        return F32
+    if v.dtype == torch.float16:
+        return F16
+    raise TypeError("v must be float32 or float16")
+
+
+def _need_cuda(t, name):
+    if not (isinstance(t, torch.Tensor) and t.is_cuda and t.is_contiguous()):
+        raise ValueError(f"{name} must be a contiguous CUDA tensor")
+
+
+class _CudaView:
+    """Zero-copy torch view of library-owned device memory (read-only use)."""
+
+    def __init__(self, ptr, shape, typestr):
+        self.__cuda_array_interface__ = {"shape": tuple(shape), "typestr": typestr,
+                                         "data": (int(ptr), False), "version": 3, "strides": None}
+
+
+class PreparedMatrix:
+    """A weight matrix W [in_dim x out_dim] (fp16) prepared for effort_gemv."""
+
+    def __init__(self, W, keep_fraction=1.0):
+        _need_cuda(W, "W")
+        if W.dtype != torch.float16 or W.dim() != 2:
+            raise ValueError("W must be a 2-D float16 tensor")
+        self.in_dim, self.out_dim = W.shape
+        self.device = W.device
+        self.keep_fraction = float(keep_fraction)
+        h = ctypes.c_void_p()
+        with torch.cuda.device(W.device):
+            _check(lib().effort_prepare(_ptr(W), self.in_dim, self.out_dim, ctypes.c_float(keep_fraction),
+                                        _stream(W.device), ctypes.byref(h)), "effort_prepare")
+        self._h = h
+
+    def gemv(self, v, effort, out=None, cutoff=None, count=None, rowlen=None):
+        """out[j] = sum over used (i, j) of v[i] * W[i, j]; returns out (fp32)."""
+        _need_cuda(v, "v")
+        if v.shape != (self.in_dim,):
+            raise ValueError("v has the wrong shape")
+        if out is None:
+            out = torch.empty(self.out_dim, device=v.device, dtype=torch.float32)
+        _need_cuda(out, "out")
+        if out.dtype != torch.float32 or out.shape != (self.out_dim,):
+            raise ValueError("out must be float32 [out_dim]")
+        for t, dt, shp, nm in ((cutoff, torch.float32, (1,), "cutoff"), (count, torch.int64, (1,), "count"),
+                               (rowlen, torch.int32, (self.in_dim,), "rowlen")):
+            if t is not None:
+                _need_cuda(t, nm)
+                if t.dtype != dt or tuple(t.shape) != shp:
+                    raise ValueError(f"{nm} must be {dt} of shape {shp}")
+        _check(lib().effort_gemv_ex(self._h, _ptr(v), _vdtype(v), ctypes.c_float(effort), _ptr(out), _ptr(cutoff),
+                                    _ptr(count), _ptr(rowlen), _stream(v.device)), "effort_gemv")
+        return out
+
+    def check(self):
+        _check(lib().effort_check(self._h), "effort_check")
+
+    def info(self):
+        i, o = ctypes.c_int64(), ctypes.c_int64()
+        k, b = ctypes.c_float(), ctypes.c_size_t()
+        _check(lib().effort_get_info(self._h, ctypes.byref(i), ctypes.byref(o), ctypes.byref(k), ctypes.byref(b)),
+               "effort_get_info")
+        return {"in_dim": i.value, "out_dim": o.value, "keep_fraction": k.value, "device_bytes": b.value}
+
+    def layout(self):
+        """Device storage as read-only torch views (for format checks)."""
+        L = Layout()
+        _check(lib().effort_get_layout(self._h, ctypes.byref(L)), "effort_get_layout")
+        I, T, cap, C = L.in_dim, L.n_tiles, L.bucket_cap, L.n_ck
+
+        def view(ptr, shape, typestr):
+            return torch.as_tensor(_CudaView(ptr, shape, typestr), device=self.device)
+
+        return {
+            "n_kept": L.n_kept, "n_tiles": T, "bucket_cap": cap, "ck_step": L.ck_step, "n_ck": C,
+            "vals": view(L.vals, (T, I, cap), "<i2"), "idx": view(L.idx, (T, I, cap), "|u1"),
+            "probes": view(L.probes, (I, L.n_probes), "<i2"), "ckmag": view(L.ckmag, (I, C + 1), "<i2"),
+            "cnt": view(L.cnt, (I, C, T), "|u1"), "wdense": view(L.wdense, (I, T * 256), "<i2"),
+            "rec": view(L.rec, (L.n_groups, 64, 4), "<u4"), "gcnt": view(L.gcnt, (L.n_groups,), "<u4"),
+        }
+
+    def close(self):
+        if getattr(self, "_h", None):
+            lib().effort_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+class Workspace:
+    """Scratch for batched and dense calls on in_dim x out_dim matrices."""
+
+    def __init__(self, in_dim, out_dim, max_pairs=1, device=None):
+        self.in_dim, self.out_dim, self.max_pairs = int(in_dim), int(out_dim), int(max_pairs)
+        h = ctypes.c_void_p()
+        with torch.cuda.device(device if device is not None else torch.cuda.current_device()):
+            _check(lib().effort_workspace_create(self.in_dim, self.out_dim, self.max_pairs, ctypes.byref(h)),
+                   "effort_workspace_create")
+        self._h = h
+
+    def close(self):
+        if getattr(self, "_h", None):
+            lib().effort_workspace_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def gemv_batched(ws, mats, hidx, vidx, V, efforts, OUT=None, cutoffs=None, counts=None):
+    """Independent matvecs: pair p uses mats[hidx[p]] on V[vidx[p]] at efforts[p] -> OUT[p]."""
+    _need_cuda(V, "V")
+    n = len(hidx)
+    if not (len(vidx) == n and len(efforts) == n):
+        raise ValueError("hidx, vidx and efforts must have the same length")
+    if OUT is None:
+        OUT = torch.empty(n, ws.out_dim, device=V.device, dtype=torch.float32)
+    handles = (ctypes.c_void_p * len(mats))(*[m._h.value for m in mats])
+    hi = (ctypes.c_int32 * n)(*[int(x) for x in hidx])
+    vi = (ctypes.c_int32 * n)(*[int(x) for x in vidx])
+    ef = (ctypes.c_float * n)(*[float(x) for x in efforts])
+    if any(not (0 <= int(x) < len(mats)) for x in hidx) or any(not (0 <= int(x) < V.shape[0]) for x in vidx):
+        raise ValueError("hidx / vidx out of range")
+    _check(lib().effort_gemv_batched(ws._h, handles, hi, vi, n, _ptr(V), _vdtype(V), ef, _ptr(OUT), _ptr(cutoffs),
+                                     _ptr(counts), _stream(V.device)), "effort_gemv_batched")
+    return OUT
+
+
+def dense_gemv(ws, W, v, out=None):
+    """Dense baseline out = W^T v with the library's streaming kernel."""
+    _need_cuda(W, "W")
+    _need_cuda(v, "v")
+    if out is None:
+        out = torch.empty(W.shape[1], device=W.device, dtype=torch.float32)
+    _check(lib().effort_dense_gemv(ws._h, _ptr(W), W.shape[0], W.shape[1], _ptr(v), _vdtype(v), _ptr(out),
+                                   _stream(W.device)), "effort_dense_gemv")
+    return out

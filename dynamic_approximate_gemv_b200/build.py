@@ -1,0 +1,54 @@
+"""Builds libeffort.so in-tree with nvcc for sm_100a (B200).
+
+Run as ``python -m dynamic_approximate_gemv_b200.build``; ``__graft_entry__``
+calls :func:`build`.  Device code is compiled without fast-math and with
+denormals kept, so the selection products round exactly as the C ABI states.
+"""
+import os
+import subprocess
+import sys
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+CSRC = os.path.join(HERE, "csrc")
+LIB = os.path.join(HERE, "libeffort.so")
+SOURCES = ["api.cu", "prep.cu", "cutoff.cu", "mac.cu", "dense.cu"]
+NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
+
+FLAGS = [
+    "-gencode", "arch=compute_100a,code=sm_100a",
+    "-O3", "-lineinfo", "-std=c++17",
+    "-shared", "-Xcompiler", "-fPIC", "-Xcompiler", "-ffp-contract=off",
+    "-ftz=false", "-prec-div=true", "-prec-sqrt=true",
+    "-Xptxas", "-v",
+]
+
+
+def needs_build():
+    if not os.path.exists(LIB):
+        return True
+    t = os.path.getmtime(LIB)
+    deps = [os.path.join(CSRC, f) for f in os.listdir(CSRC)] + [
+        os.path.join(HERE, "..", "include", "effort.h"), __file__]
+    return any(os.path.getmtime(p) > t for p in deps if os.path.exists(p))
+
+
+def build(force=False, verbose=False):
+    """Compile the CUDA sources into libeffort.so next to this file."""
+    if not force and not needs_build():
+        return LIB
+    cmd = [NVCC] + FLAGS + ["-I" + os.path.join(HERE, "..", "include"), "-o", LIB + ".tmp"] + [
+        os.path.join(CSRC, s) for s in SOURCES]
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    log = res.stdout + res.stderr
+    with open(os.path.join(HERE, "build.log"), "w") as f:
+        f.write(" ".join(cmd) + "\n" + log)
+    if res.returncode != 0:
+        raise RuntimeError("nvcc failed:\n" + log[-8000:])
+    os.replace(LIB + ".tmp", LIB)
+    if verbose:
+        print(log)
+    return LIB
+
+
+if __name__ == "__main__":
+    build(force="--force" in sys.argv, verbose=True)

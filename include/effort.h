@@ -1,0 +1,192 @@
+/*
+ * effort.h -- C ABI of the B200 (sm_100a) library for the "Effort"
+ * approximate matrix-vector multiply.
+ *
+ * The method (Hacker News item 40067677, "Show HN: Speeding up LLM inference
+ * 2x times (possibly)", the pseudo-code quoted in a commenter's question and
+ * the author's replies): every row of the weight matrix is stored sorted by
+ * |w| descending; per call, an input vector v and an effort in (0, 1] pick a
+ * cutoff c from per-row probes (cutoff_chart = v * probes, cutoff =
+ * topK(chart, effort)), and only the products with |v_i| * |w_ij| >= c are
+ * multiplied and added.  The author's complexity reply (Hacker News item
+ * 40095016) gives O(effort * inDim * outDim) multiplications, O(inDim) for the
+ * dispatch and about O(inDim log inDim) for the cutoff.
+ *
+ * Conventions (all entry points):
+ *  - W is [in_dim x out_dim] binary16, row-major: row i holds the weights that
+ *    multiply v[i], and out[j] = sum_i v[i] * W[i][j] (the matrix is already
+ *    "flipped" in the sense of the pages).
+ *  - Pointers named W, v, V, out, OUT, *_out are DEVICE pointers unless stated.
+ *    The caller owns them; the library never frees them.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *  - Every call returns an effort_status_t.  Argument errors are detected on
+ *    the host before anything is launched.  No exception or abort crosses the
+ *    ABI.  Device faults are never used to signal errors.
+ *  - Selection rule: a kept pair (i, j) is used iff the single-precision
+ *    product fl32(|v_i| * |w_ij|) (round to nearest even, no FMA, no flush to
+ *    zero) is >= c.  Ties at c are used.  Outputs are accumulated in fp32.
+ */
+#ifndef EFFORT_H
+#define EFFORT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct effort_handle_s* effort_handle_t;        /* prepared matrix, library-owned */
+typedef struct effort_workspace_s* effort_workspace_t;  /* per-call scratch, library-owned */
+
+typedef enum {
+  EFFORT_OK = 0,
+  EFFORT_ERR_ARG = 1,          /* bad pointer, size, effort, keep fraction or dtype */
+  EFFORT_ERR_CUDA = 2,         /* a CUDA runtime call or kernel launch failed */
+  EFFORT_ERR_NOMEM = 3,        /* device or host allocation failed */
+  EFFORT_ERR_NONFINITE = 4,    /* W (prepare) or v (reported by effort_check) held inf/NaN */
+  EFFORT_ERR_DEVICE = 5,       /* a kernel reported an internal inconsistency */
+  EFFORT_ERR_UNSUPPORTED = 6   /* sizes outside the limits stated below */
+} effort_status_t;
+
+typedef enum { EFFORT_F32 = 0, EFFORT_F16 = 1 } effort_dtype_t;
+
+/* Size limits of this build. */
+#define EFFORT_MAX_OUT_DIM 32768      /* a row is sorted inside one thread block */
+#define EFFORT_MAX_IN_DIM 40960       /* the cutoff's chart lives in one cluster's shared memory */
+#define EFFORT_MAX_PAIRS_PER_LAUNCH 16
+
+/*
+ * effort_prepare -- the offline pass: `precompute(W)` of the pages.
+ *   Sorts every row of W by |w| descending (ties: lower column first), keeps
+ *   the first n = floor(keep_fraction * out_dim + 1/2) entries of each row
+ *   (the post text: the format lets the loader skip the least important
+ *   weights), takes 16 midpoint-rank probes per row, and stores the kept
+ *   entries in output-tile buckets of 256 columns (fp16 value + 8-bit local
+ *   index, bucket-sorted by |w|), a dense copy of the kept weights, and the
+ *   checkpoint tables the dispatch uses.
+ *   W: device, binary16 [in_dim x out_dim], 2-byte aligned; read only during
+ *      the call (the stream is synchronised before returning; the caller may
+ *      free W afterwards).
+ *   keep_fraction: (0, 1].  Must keep at least one weight per row.
+ *   Limits: 1 <= out_dim <= EFFORT_MAX_OUT_DIM, 1 <= in_dim <= EFFORT_MAX_IN_DIM,
+ *           in_dim * out_dim < 2^32.
+ *   Returns EFFORT_ERR_NONFINITE (and no handle) if W holds inf or NaN.
+ *   On success *out_handle owns all device storage; free it with effort_destroy.
+ */
+effort_status_t effort_prepare(const void* W, int64_t in_dim, int64_t out_dim, float keep_fraction,
+                               void* stream, effort_handle_t* out_handle);
+
+/*
+ * effort_gemv -- one approximate matvec: `approxMul(v, ...)` of the pages.
+ *   v: device fp32 [in_dim]; out: device fp32 [out_dim], fully overwritten.
+ *   effort in (0, 1]: K = llround(effort * in_dim * out_dim) products are
+ *   targeted; the cutoff c is the weighted K-th largest entry of the chart
+ *   fl32(|v_i| * probe_ik) (c = 0 if K >= the kept count, c = +inf if K = 0).
+ *   Asynchronous and stream-ordered: no host synchronisation and no
+ *   allocation; two kernels (cutoff+dispatch, then multiply-accumulate).
+ *   A handle holds one call's scratch: calls on the same handle must be
+ *   ordered (same stream, or synchronised); concurrent calls on one handle race.
+ */
+effort_status_t effort_gemv(effort_handle_t h, const float* v, float effort, float* out, void* stream);
+
+/*
+ * effort_gemv_ex -- effort_gemv with a v dtype and optional device outputs.
+ *   v: device, EFFORT_F32 or EFFORT_F16, [in_dim].
+ *   cutoff_out: nullable device float, receives c.
+ *   count_out: nullable device uint64, receives |S|, the number of used products.
+ *   rowlen_out: nullable device uint32 [in_dim], receives L_i, the number of
+ *     used products of row i (always a leading part of row i's sorted order).
+ */
+effort_status_t effort_gemv_ex(effort_handle_t h, const void* v, effort_dtype_t v_dtype, float effort,
+                               float* out, float* cutoff_out, uint64_t* count_out, uint32_t* rowlen_out,
+                               void* stream);
+
+/*
+ * effort_check -- synchronises the handle's last stream and reports whether a
+ *   call since the previous check saw a non-finite entry of v
+ *   (EFFORT_ERR_NONFINITE; those calls' outputs are unspecified) or an internal
+ *   device inconsistency (EFFORT_ERR_DEVICE).  Clears the flags.
+ */
+effort_status_t effort_check(effort_handle_t h);
+
+/*
+ * Workspaces: scratch for effort_gemv_batched and effort_dense_gemv.
+ *   Sized for matrices of in_dim x out_dim and up to max_pairs concurrent pairs
+ *   per call (max_pairs >= 1).  Allocates device memory (not stream-ordered).
+ */
+effort_status_t effort_workspace_create(int64_t in_dim, int64_t out_dim, int32_t max_pairs,
+                                        effort_workspace_t* out_ws);
+effort_status_t effort_workspace_destroy(effort_workspace_t ws);
+
+/*
+ * effort_gemv_batched -- n_pairs independent matvecs (MoE-style routing: each
+ *   vector meets the experts it was routed to; the author's complexity reply
+ *   likens the per-multiplication choice of buckets to expert routing).
+ *   Pair p uses handles[hidx[p]], vector V + vidx[p] * in_dim (dtype v_dtype),
+ *   efforts[p], and writes OUT + p * out_dim (fp32).  hidx, vidx, efforts:
+ *   HOST arrays of n_pairs entries.  All handles must share in_dim/out_dim
+ *   with the workspace.  cutoffs_out [n_pairs] float and counts_out
+ *   [n_pairs] uint64 are nullable device arrays.  One cutoff per pair.
+ *   Launches two kernels per group of up to EFFORT_MAX_PAIRS_PER_LAUNCH pairs.
+ *   n_pairs <= the workspace's max_pairs.
+ */
+effort_status_t effort_gemv_batched(effort_workspace_t ws, const effort_handle_t* handles, const int32_t* hidx,
+                                    const int32_t* vidx, int32_t n_pairs, const void* V, effort_dtype_t v_dtype,
+                                    const float* efforts, float* OUT, float* cutoffs_out, uint64_t* counts_out,
+                                    void* stream);
+
+/*
+ * effort_dense_gemv -- the dense baseline out = W^T v (every weight, fp32
+ *   accumulation), hand-written streaming kernel.  W: device binary16
+ *   [in_dim x out_dim], out_dim a multiple of 8, 16-byte aligned.  v: fp32 or
+ *   fp16 [in_dim].  Uses the workspace's first pair slot.
+ */
+effort_status_t effort_dense_gemv(effort_workspace_t ws, const void* W, int64_t in_dim, int64_t out_dim,
+                                  const void* v, effort_dtype_t v_dtype, float* out, void* stream);
+
+/* Sizes and footprint of a prepared matrix. */
+effort_status_t effort_get_info(effort_handle_t h, int64_t* in_dim, int64_t* out_dim, float* keep_fraction,
+                                size_t* device_bytes);
+
+/*
+ * effort_layout_t -- read-only view of a handle's device storage, for format
+ * checks.  Bucket (i, t) holds the kept entries of row i with columns in
+ * [256 t, 256 t + 256), sorted by |w| descending (ties: lower column), at
+ * entry offset (t * in_dim + i) * bucket_cap of `vals` (binary16 bits) and
+ * `idx` (column - 256 t); unused slots hold +0.0 / 0.
+ * probes: [in_dim][16] |w| binary16 bits at the probe ranks (0 for empty segments).
+ * ckmag: [in_dim][n_ck + 1]: [0] = |w| at rank 0; [1 + k] = |w| at rank
+ *   min((k + 1) * ck_step, n) - 1.
+ * cnt: [in_dim][n_ck][n_tiles] uint8: entries of tile t among the first
+ *   min((k + 1) * ck_step, n) ranks of row i, saturated at 255.
+ * wdense: [in_dim][n_tiles * 256] binary16: kept weights at their columns, 0 elsewhere.
+ * rec / gcnt: the last call's dispatch records (see the library source).
+ */
+typedef struct {
+  int64_t in_dim, out_dim;
+  int32_t n_kept, n_tiles, bucket_cap, ck_step, n_ck, n_probes;
+  const void* vals;
+  const void* idx;
+  const void* probes;
+  const void* ckmag;
+  const void* cnt;
+  const void* wdense;
+  const void* rec;
+  const void* gcnt;
+  int32_t n_groups;
+} effort_layout_t;
+
+effort_status_t effort_get_layout(effort_handle_t h, effort_layout_t* layout);
+
+/* Frees the handle's device storage after synchronising its last stream. */
+effort_status_t effort_destroy(effort_handle_t h);
+
+/* Static string naming a status code. */
+const char* effort_status_string(effort_status_t s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EFFORT_H */

@@ -1,0 +1,273 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Contract per call, on seeded synthetic inputs:
+  * the cutoff c equals the oracle's bit for bit;
+  * the used set for that c matches exactly: |S| and every row's used length
+    L_i equal the oracle's (used sets are leading parts of each row's sorted
+    order, and the kernel's predicate is the oracle's, so equal per-row counts
+    with no double visits mean equal sets; one-hot vectors check single rows
+    product by product);
+  * out agrees with the oracle's float64 sum over the same set to relative
+    L2 <= 1e-4 and max abs error <= 1e-3 * ||out||_inf.
+"""
+import numpy as np
+import pytest
+import torch
+
+from dynamic_approximate_gemv_b200 import inputs
+from oracle import effort_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+REL_L2 = 1e-4
+MAX_ABS = 1e-3
+
+
+@pytest.fixture(scope="module")
+def E():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from dynamic_approximate_gemv_b200 import build
+    build.build()
+    import dynamic_approximate_gemv_b200 as E
+    E.lib()
+    return E
+
+
+def f32bits(x):
+    return int(np.array([x], np.float32).view(np.uint32)[0])
+
+
+def assert_out_close(got, ref):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    nref = np.linalg.norm(ref)
+    inf = np.max(np.abs(ref)) if ref.size else 0.0
+    if nref == 0.0:
+        assert np.max(np.abs(got)) == 0.0
+        return
+    assert np.linalg.norm(got - ref) <= REL_L2 * nref, np.linalg.norm(got - ref) / nref
+    assert np.max(np.abs(got - ref)) <= MAX_ABS * inf
+
+
+def run_gpu(E, pm, v, effort):
+    I = pm.in_dim
+    dev = torch.device("cuda")
+    cutoff = torch.empty(1, device=dev, dtype=torch.float32)
+    count = torch.full((1,), -1, device=dev, dtype=torch.int64)
+    rowlen = torch.full((I,), -7, device=dev, dtype=torch.int32)
+    out = pm.gemv(v, effort, cutoff=cutoff, count=count, rowlen=rowlen)
+    torch.cuda.synchronize()
+    pm.check()
+    return float(cutoff.item()), int(count.item()), rowlen.cpu().numpy().astype(np.int64), out.cpu().numpy()
+
+
+def check_call(E, prep, pm, v_np, effort):
+    v = torch.from_numpy(v_np).cuda()
+    c, count, rowlen, out = run_gpu(E, pm, v, effort)
+    ref = O.effort_gemv(prep, v_np, effort)
+    assert f32bits(c) == f32bits(ref.c), (c, float(ref.c))
+    assert count == ref.count
+    assert np.array_equal(rowlen, ref.L)
+    assert_out_close(out, ref.out)
+    return ref
+
+
+def make(E, I, Od, seed, keep=1.0):
+    Wn = inputs.weights(I, Od, seed)
+    prep = O.Prepared(Wn.view(np.uint16), keep)
+    pm = E.PreparedMatrix(torch.from_numpy(Wn).cuda(), keep)
+    return Wn, prep, pm
+
+
+# ------------------------------------------------------------------ format
+def check_layout(prep, pm):
+    L = {k: (v.cpu().numpy() if isinstance(v, torch.Tensor) else v) for k, v in pm.layout().items()}
+    I, Od, n = prep.in_dim, prep.out_dim, prep.n
+    T, H, C = L["n_tiles"], L["ck_step"], L["n_ck"]
+    assert L["n_kept"] == n
+    Wb = prep.W_bits
+    for i in range(I):
+        order = prep.W_idx[i, :n]
+        tiles = order // 256
+        for t in range(T):
+            cols = order[tiles == t]
+            nb = cols.size
+            assert np.array_equal(L["vals"][t, i, :nb].view(np.uint16), Wb[i, cols])
+            assert np.array_equal(L["idx"][t, i, :nb], (cols - 256 * t).astype(np.uint8))
+            assert not np.any(L["vals"][t, i, nb:]) and not np.any(L["idx"][t, i, nb:])
+            for k in range(C):
+                end = min((k + 1) * H, n)
+                assert L["cnt"][i, k, t] == min(255, int(np.sum(tiles[:end] == t)))
+        mag = (Wb[i, order] & 0x7FFF)
+        ranks, weights = O.probe_layout(n)
+        exp_probes = np.where(weights > 0, mag[np.maximum(ranks, 0)], 0)
+        assert np.array_equal(L["probes"][i].view(np.uint16), exp_probes)
+        ck = [mag[0]] + [mag[min((k + 1) * H, n) - 1] for k in range(C)]
+        assert np.array_equal(L["ckmag"][i].view(np.uint16), np.array(ck, np.uint16))
+        dense = np.zeros(T * 256, np.uint16)
+        dense[order] = Wb[i, order]
+        assert np.array_equal(L["wdense"][i].view(np.uint16), dense)
+
+
+@pytest.mark.parametrize("I,Od,keep", [(40, 300, 1.0), (33, 513, 0.75), (7, 9, 1.0), (64, 1024, 0.8)])
+def test_layout_matches_oracle_order(E, I, Od, keep):
+    _, prep, pm = make(E, I, Od, 101, keep)
+    check_layout(prep, pm)
+
+
+# ------------------------------------------------------------------ parity
+@pytest.mark.parametrize("effort", [0.25, 0.15, 0.4, 0.5, 1.0, 0.05])
+def test_512_square(E, effort):
+    _, prep, pm = make(E, 512, 512, 0)
+    v = inputs.vector(512, 1)
+    check_call(E, prep, pm, v, effort)
+
+
+@pytest.mark.parametrize("I,Od,keep,dist,effort", [
+    (100, 300, 1.0, "normal", 0.25),   # ragged last tile
+    (33, 513, 0.75, "t3", 0.3),        # one-column last tile, keep < 1
+    (1, 1, 1.0, "normal", 1.0),
+    (1, 1, 1.0, "normal", 0.5),
+    (5, 7, 1.0, "t3", 0.4),
+    (2000, 700, 0.6, "t3", 0.2),
+    (777, 2049, 1.0, "normal", 0.12),
+    (64, 32768, 1.0, "normal", 0.25),  # widest supported row
+])
+def test_ragged_and_edge_shapes(E, I, Od, keep, dist, effort):
+    _, prep, pm = make(E, I, Od, 7, keep)
+    check_call(E, prep, pm, inputs.vector(I, 8, dist), effort)
+
+
+def test_tiny_effort_selects_nothing(E):
+    _, prep, pm = make(E, 64, 64, 3)
+    ref = check_call(E, prep, pm, inputs.vector(64, 4), 1e-6)
+    assert ref.count == 0 and np.isinf(ref.c)
+
+
+def test_zero_and_repeated_vector_entries(E):
+    _, prep, pm = make(E, 300, 600, 5)
+    v = inputs.vector(300, 6)
+    v[::4] = 0.0
+    v[1::7] = v[1]
+    for e in (0.1, 0.3, 0.9):
+        check_call(E, prep, pm, v, e)
+
+
+def test_all_zero_vector(E):
+    _, prep, pm = make(E, 50, 300, 9)
+    ref = check_call(E, prep, pm, np.zeros(50, np.float32), 0.3)
+    assert float(ref.c) == 0.0  # chart is all zero: every kept product (all zero) is used
+
+
+def test_fp16_vector(E):
+    _, prep, pm = make(E, 512, 768, 11)
+    v = inputs.vector(512, 12, dtype=np.float16)
+    check_call(E, prep, pm, v, 0.25)
+
+
+def test_one_hot_rows_product_by_product(E):
+    Wn, prep, pm = make(E, 64, 700, 13)
+    for i in (0, 17, 63):
+        v = np.zeros(64, np.float32)
+        v[i] = -1.7
+        ref = O.effort_gemv(prep, v, 0.004)
+        out = pm.gemv(torch.from_numpy(v).cuda(), 0.004).cpu().numpy()
+        w = Wn[i].astype(np.float32)
+        exp = np.where(ref.mask[i], (np.float32(-1.7) * w).astype(np.float32), 0.0)
+        assert np.array_equal(out, exp.astype(np.float32))
+
+
+def test_repeat_calls_are_deterministic(E):
+    _, prep, pm = make(E, 1024, 1536, 14)
+    v = torch.from_numpy(inputs.vector(1024, 15, "t3")).cuda()
+    first = pm.gemv(v, 0.25).clone()
+    for _ in range(5):
+        assert torch.equal(pm.gemv(v, 0.25), first)
+
+
+def test_effort_sweep_4096_square(E):
+    _, prep, pm = make(E, 4096, 4096, 2)
+    v = inputs.vector(4096, 3, dtype=np.float16)
+    refs = [check_call(E, prep, pm, v, e) for e in (1.0, 0.5, 0.4, 0.25, 0.15)]
+    counts = [r.count for r in refs]
+    assert counts == sorted(counts, reverse=True)
+
+
+@pytest.mark.parametrize("I,Od,keep,effort", [(4096, 14336, 1.0, 0.25), (14336, 4096, 1.0, 0.25),
+                                             (4096, 14336, 0.75, 0.15)])
+def test_ffn_shapes_full_size(E, I, Od, keep, effort):
+    _, prep, pm = make(E, I, Od, 4, keep)
+    check_call(E, prep, pm, inputs.vector(I, 7, "t3"), effort)
+
+
+def test_nonfinite_inputs_are_reported(E):
+    Wn = inputs.weights(16, 32, 1)
+    Wn[3, 5] = np.float16(np.inf)
+    with pytest.raises(E.EffortError) as ei:
+        E.PreparedMatrix(torch.from_numpy(Wn).cuda())
+    assert ei.value.status == 4
+    _, prep, pm = make(E, 16, 32, 2)
+    v = inputs.vector(16, 3)
+    v[2] = np.nan
+    pm.gemv(torch.from_numpy(v).cuda(), 0.5)
+    with pytest.raises(E.EffortError) as ei:
+        pm.check()
+    assert ei.value.status == 4
+    pm.check()  # the flag is cleared
+
+
+def test_argument_errors(E):
+    _, _, pm = make(E, 16, 32, 2)
+    v = torch.zeros(16, device="cuda")
+    for bad in (0.0, 1.5, float("nan"), -1.0):
+        with pytest.raises(E.EffortError):
+            pm.gemv(v, bad)
+
+
+# ------------------------------------------------------------------ batched / MoE
+def test_batched_pairs_match_single_calls(E):
+    I, Od = 512, 1024
+    mats, preps = [], []
+    for x in range(3):
+        Wn = inputs.weights(I, Od, 100 + x)
+        preps.append(O.Prepared(Wn.view(np.uint16), 1.0))
+        mats.append(E.PreparedMatrix(torch.from_numpy(Wn).cuda()))
+    V = np.stack([inputs.vector(I, 200 + k) for k in range(4)])
+    hidx = [0, 2, 1, 2, 0, 1, 2]
+    vidx = [0, 0, 1, 1, 2, 3, 3]
+    eff = [0.5, 0.25, 0.12, 0.25, 1.0, 0.4, 0.05]
+    ws = E.Workspace(I, Od, max_pairs=len(hidx))
+    Vt = torch.from_numpy(V).cuda()
+    cut = torch.empty(len(hidx), device="cuda")
+    cnt = torch.zeros(len(hidx), device="cuda", dtype=torch.int64)
+    OUT = E.gemv_batched(ws, mats, hidx, vidx, Vt, eff, cutoffs=cut, counts=cnt)
+    torch.cuda.synchronize()
+    for p in range(len(hidx)):
+        ref = O.effort_gemv(preps[hidx[p]], V[vidx[p]], eff[p])
+        assert f32bits(cut[p].item()) == f32bits(ref.c)
+        assert int(cnt[p].item()) == ref.count
+        assert_out_close(OUT[p].cpu().numpy(), ref.out)
+
+
+def test_batched_more_pairs_than_one_launch(E):
+    I, Od = 256, 512
+    Wn = inputs.weights(I, Od, 300)
+    prep = O.Prepared(Wn.view(np.uint16), 1.0)
+    m = E.PreparedMatrix(torch.from_numpy(Wn).cuda())
+    n = 37
+    V = np.stack([inputs.vector(I, 400 + k) for k in range(n)])
+    ws = E.Workspace(I, Od, max_pairs=n)
+    OUT = E.gemv_batched(ws, [m], [0] * n, list(range(n)), torch.from_numpy(V).cuda(), [0.25] * n)
+    for p in (0, 15, 16, 36):
+        assert_out_close(OUT[p].cpu().numpy(), O.effort_gemv(prep, V[p], 0.25).out)
+
+
+# ------------------------------------------------------------------ dense baseline
+@pytest.mark.parametrize("I,Od", [(512, 512), (100, 296), (4096, 4096)])
+def test_dense_gemv(E, I, Od):
+    Wn = inputs.weights(I, Od, 21)
+    v = inputs.vector(I, 22)
+    ws = E.Workspace(I, Od)
+    out = E.dense_gemv(ws, torch.from_numpy(Wn).cuda(), torch.from_numpy(v).cuda()).cpu().numpy()
+    assert_out_close(out, O.dense_gemv(Wn.view(np.uint16), v))
