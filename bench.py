@@ -1,0 +1,464 @@
+#!/usr/bin/env python
+"""Benchmark of the Effort approximate GEMV on B200.
+
+Headline workload: one approximate matvec out = W^T v with W 4096 x 14336 fp16
+(Mistral-7B FFN w1/w3 shape, entries N(0, 0.02^2)), v fp32 Student-t(3) /
+sqrt(3), effort 0.25, keep 1.0, batch 1.  A step is one call of the library's
+gemv (cutoff + dispatch kernel, then multiply kernel) on inputs resident in
+HBM.  Steps rotate over 10 prepared matrices and 8 vectors, so the bytes a
+call reads are not in L2 from the previous use.  Steps are issued from CUDA
+graphs (Python launch overhead would otherwise dominate a ~10 us call).
+
+Prints ONE JSON line (rank 0).  `--impl reference` times the CPU oracle
+instead (the reference arm).  `--gpus N` under torchrun runs N independent
+replicas (the path is single-GPU; no collective on the data path).
+"""
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "approx-GEMV µs & achieved HBM GB/s vs effort (4096×14336 fp16, batch 1)"
+IN_DIM, OUT_DIM = 4096, 14336
+EFFORT, KEEP = 0.25, 1.0
+N_MATS, N_VECS, GRAPH_STEPS = 10, 8, 40
+SWEEP = (1.0, 0.5, 0.4, 0.25, 0.15)
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+CPU_SAMPLE_ROWS = 256
+
+
+def args_parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--ncu", action="store_true",
+                    help="small profiling case: 4 prepared matrices, 8 warm calls then 4 calls, no timing")
+    return ap.parse_args()
+
+
+def hbm_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def workload_config():
+    return {"workload": f"approx GEMV W {IN_DIM}x{OUT_DIM} fp16 N(0,0.02^2), v fp32 t3/sqrt(3), "
+                        f"effort {EFFORT}, keep {KEEP}, batch 1",
+            "in_dim": IN_DIM, "out_dim": OUT_DIM, "effort": EFFORT, "keep_fraction": KEEP,
+            "l2": f"inputs larger than L2: {N_MATS} prepared matrices x {N_VECS} vectors rotated",
+            "issue": f"CUDA graphs of {GRAPH_STEPS} steps"}
+
+
+# ----------------------------------------------------------------- CPU oracle
+def oracle_sample(seed=4):
+    """A CPU_SAMPLE_ROWS-row slice of the headline workload, prepared for the oracle."""
+    from dynamic_approximate_gemv_b200 import inputs
+    from oracle import effort_oracle as O
+    Wn = inputs.weights(CPU_SAMPLE_ROWS, OUT_DIM, seed)
+    prep = O.Prepared(Wn.view(np.uint16), KEEP)
+    vs = [inputs.vector(CPU_SAMPLE_ROWS, 50 + k, "t3") for k in range(4)]
+    return prep, vs
+
+
+def time_oracle(steps, warmup, min_seconds=0.0):
+    """Oracle matvecs on the row slice; returns us per full matvec (scaled by rows)."""
+    from oracle import effort_oracle as O
+    prep, vs = oracle_sample()
+    for k in range(warmup):
+        O.effort_gemv(prep, vs[k % len(vs)], EFFORT)
+    t0 = time.perf_counter()
+    done = 0
+    while done < steps or (time.perf_counter() - t0) < min_seconds:
+        O.effort_gemv(prep, vs[done % len(vs)], EFFORT)
+        done += 1
+    dt = time.perf_counter() - t0
+    scale = IN_DIM / CPU_SAMPLE_ROWS
+    return dt / done * scale * 1e6, done, dt
+
+
+def cpu_baseline_record(us, done, dt):
+    return {"value": us, "unit": "us", "cores": 1, "kind": "oracle",
+            "sample": f"{done} oracle matvecs on a {CPU_SAMPLE_ROWS}x{OUT_DIM} row slice of the workload "
+                      f"({dt:.1f} s), time scaled by {IN_DIM // CPU_SAMPLE_ROWS} to the full matvec; "
+                      f"numpy, single thread"}
+
+
+def run_reference(a):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    us, done, dt = time_oracle(a.steps, a.warmup)
+    line = {"metric": METRIC, "value": us, "unit": "us", "n_gpus": a.gpus, "steps": a.steps, "warmup": a.warmup,
+            "ms_per_step": us / 1000.0, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic", "impl": "reference", "config": workload_config(),
+            "cpu_baseline": cpu_baseline_record(us, done, dt),
+            "e2e": {"value": us, "unit": "us", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.file, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.file.flush()
+        rows = []
+        with open(self.file.name) as f:
+            for line in f:
+                p = [x.strip() for x in line.split(",")]
+                if len(p) < 9:
+                    continue
+                try:
+                    rows.append((float(p[1]), float(p[2]), float(p[3]), p[5:9]))
+                except ValueError:
+                    continue
+        os.unlink(self.file.name)
+        if not rows:
+            return None
+        pmax = max(r[2] for r in rows)
+        load = [r for r in rows if r[2] >= 0.5 * pmax] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in load for k in range(4) if r[3][k].lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in load), "sm_max_mhz": max(r[1] for r in load),
+                "reasons": reasons, "samples": len(load), "power_w_max": pmax}
+
+
+# ----------------------------------------------------------------- GPU arm
+def source_sha(*names):
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "dynamic_approximate_gemv_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel):
+    """DRAM bytes per launch from the committed ncu summary, if its source hash is current."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            rec = json.load(f)[kernel]
+        if rec["source_sha"] != source_sha(*rec["sources"]):
+            return None
+        return float(rec["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+def run_ncu_case():
+    """Plain launches for an ncu capture: the headline shape, 4 matrices rotated
+    (each call reads ~50 MB of a 330 MB prepared matrix; 4 x 50 MB > L2)."""
+    import torch
+    from dynamic_approximate_gemv_b200 import build, inputs
+    build.build()
+    import dynamic_approximate_gemv_b200 as E
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev)
+    mats = []
+    for m in range(4):
+        g.manual_seed(1000 + m)
+        W = (torch.randn(IN_DIM, OUT_DIM, device=dev, generator=g) * 0.02).to(torch.float16)
+        mats.append(E.PreparedMatrix(W, KEEP))
+        del W
+    vecs = [torch.from_numpy(inputs.vector(IN_DIM, 7 + k, "t3")).to(dev) for k in range(4)]
+    out = torch.empty(OUT_DIM, device=dev)
+    for k in range(12):
+        mats[k % 4].gemv(vecs[k % 4], EFFORT, out=out)
+    torch.cuda.synchronize()
+    print("ncu case done", float(out.abs().sum()))
+
+
+def main():
+    a = args_parse()
+    if a.impl == "reference":
+        run_reference(a)
+        return
+    if a.ncu:
+        run_ncu_case()
+        return
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+
+    from dynamic_approximate_gemv_b200 import build, inputs
+    if rank == 0:
+        build.build()
+    if world > 1:
+        dist.barrier()
+    import dynamic_approximate_gemv_b200 as E
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    g = torch.Generator(device=dev)
+    mats, raws = [], []
+    for m in range(N_MATS):
+        g.manual_seed(1000 * (rank + 1) + m)
+        W = (torch.randn(IN_DIM, OUT_DIM, device=dev, generator=g) * 0.02).to(torch.float16)
+        mats.append(E.PreparedMatrix(W, KEEP))
+        raws.append(W)
+    vecs = [torch.from_numpy(inputs.vector(IN_DIM, 7 + k, "t3")).to(dev) for k in range(N_VECS)]
+    outs = [torch.empty(OUT_DIM, device=dev) for _ in range(N_MATS)]
+    torch.cuda.synchronize()
+
+    def step_pairs(n, offset=0):
+        return [((offset + k) % N_MATS, (offset + k) % N_VECS) for k in range(n)]
+
+    # used-product counts of the rotation at each effort (algorithmic bytes)
+    def mean_count(effort):
+        cnt = torch.zeros(1, device=dev, dtype=torch.int64)
+        tot = 0
+        pairs = step_pairs(GRAPH_STEPS)
+        for (mi, vi) in pairs:
+            mats[mi].gemv(vecs[vi], effort, out=outs[mi], count=cnt)
+            tot += int(cnt.item())
+        return tot / len(pairs)
+
+    def capture(n_steps, effort, offset=0):
+        gr = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream(device=dev)
+        s.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(s):
+            for (mi, vi) in step_pairs(n_steps, offset):  # warm once outside capture
+                mats[mi].gemv(vecs[vi], effort, out=outs[mi])
+        torch.cuda.current_stream(dev).wait_stream(s)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(gr, stream=s):
+            for (mi, vi) in step_pairs(n_steps, offset):
+                mats[mi].gemv(vecs[vi], effort, out=outs[mi])
+        torch.cuda.synchronize()
+        return gr
+
+    def timed_steps(effort, steps, warmup, sampler=None, min_seconds=0.0):
+        full = capture(GRAPH_STEPS, effort)
+        rem = steps % GRAPH_STEPS
+        tail = capture(rem, effort, offset=0) if rem else None
+        for _ in range(max(1, math.ceil(warmup / GRAPH_STEPS))):
+            full.replay()
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps // GRAPH_STEPS):
+            full.replay()
+        if tail is not None:
+            tail.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        barrier()
+        ms = max_over_ranks(e0.elapsed_time(e1))
+        # keep the same replay running until the clock sampler has a window of samples
+        if sampler is not None and min_seconds > 0:
+            t0 = time.perf_counter()
+            while time.perf_counter() - t0 < min_seconds:
+                for _ in range(50):
+                    full.replay()
+                torch.cuda.synchronize()
+        return ms
+
+    peak, peak_kind = hbm_peak()
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    ms = timed_steps(EFFORT, a.steps, a.warmup, sampler, min_seconds=2.0)
+    clocks = sampler.stop()
+    us_per_step = ms * 1000.0 / a.steps
+    value = us_per_step / world  # whole job: all ranks' matvecs over the max-rank time
+
+    # per-kernel durations (events between the two kernels), same rotation and effort
+    n_ph = GRAPH_STEPS
+    s = torch.cuda.Stream(device=dev)
+    evA = [torch.cuda.Event(enable_timing=True) for _ in range(n_ph + 1)]
+    evB = [torch.cuda.Event(enable_timing=True) for _ in range(n_ph)]
+    for ev in evB:
+        ev.record(s)  # creates the CUDA events the library records into
+    torch.cuda.synchronize()
+
+    def phase_pass():
+        with torch.cuda.stream(s):
+            for k, (mi, vi) in enumerate(step_pairs(n_ph)):
+                evA[k].record(s)
+                mats[mi].gemv_split(vecs[vi], EFFORT, outs[mi], evB[k], stream=s)
+            evA[n_ph].record(s)
+        torch.cuda.synchronize()
+
+    for _ in range(3):
+        phase_pass()
+    cut_ms, mac_ms = [], []
+    for _ in range(5):
+        phase_pass()
+        cut_ms += [evA[k].elapsed_time(evB[k]) for k in range(n_ph)]
+        mac_ms += [evB[k].elapsed_time(evA[k + 1]) for k in range(n_ph)]
+    mac_us = statistics.mean(mac_ms) * 1000.0
+    cut_us = statistics.mean(cut_ms) * 1000.0
+
+    S_mean = mean_count(EFFORT)
+    alg_bytes = 3.0 * S_mean + 4.0 * IN_DIM + 4.0 * OUT_DIM  # F3 bytes of the used set + v + out
+    achieved = alg_bytes / (mac_us * 1e-6) / 1e9
+    traffic = ncu_traffic("k_mac")
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                "traffic": traffic, "kernel": "k_mac", "peak_kind": peak_kind,
+                "frac_of_nominal_8000": achieved / NOMINAL_HBM_GBS,
+                "algorithmic_bytes_per_launch": alg_bytes, "launch_us": mac_us}
+
+    # dense baselines on the same rotation (raw fp16 matrices, 117 MB each)
+    ws = E.Workspace(IN_DIM, OUT_DIM)
+    vec16 = [v.to(torch.float16) for v in vecs]
+    dense_outs = [torch.empty(OUT_DIM, device=dev) for _ in range(N_MATS)]
+    mv_outs = [torch.empty(OUT_DIM, device=dev, dtype=torch.float16) for _ in range(N_MATS)]
+
+    def time_graph(fn, n_rep=20):
+        gr = torch.cuda.CUDAGraph()
+        st = torch.cuda.Stream(device=dev)
+        st.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(st):
+            fn()
+        torch.cuda.synchronize()
+        with torch.cuda.graph(gr, stream=st):
+            fn()
+        for _ in range(3):
+            gr.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(n_rep):
+            gr.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / n_rep
+
+    def dense_all():
+        for k in range(GRAPH_STEPS):
+            E.dense_gemv(ws, raws[k % N_MATS], vecs[k % N_VECS], out=dense_outs[k % N_MATS])
+
+    def mv_all():
+        for k in range(GRAPH_STEPS):
+            torch.mv(raws[k % N_MATS].t(), vec16[k % N_VECS], out=mv_outs[k % N_MATS])
+
+    dense_us = time_graph(dense_all) * 1000.0 / GRAPH_STEPS
+    mv_us = time_graph(mv_all) * 1000.0 / GRAPH_STEPS
+    dense_bytes = 2.0 * IN_DIM * OUT_DIM + 4.0 * IN_DIM + 4.0 * OUT_DIM
+    baselines = {"dense_roofline_us_measured_peak": dense_bytes / (peak * 1e9) * 1e6,
+                 "dense_roofline_us_nominal_8000": dense_bytes / (NOMINAL_HBM_GBS * 1e9) * 1e6,
+                 "k_dense_gemv_us": dense_us, "k_dense_gemv_gbs": dense_bytes / (dense_us * 1e-6) / 1e9,
+                 "torch_mv_cublas_us": mv_us}
+
+    sweep = {}
+    if not a.no_sweep:
+        for e in SWEEP:
+            msw = timed_steps(e, 400, 80)
+            us = msw * 1000.0 / 400
+            Se = mean_count(e)
+            b = 3.0 * Se + 4.0 * IN_DIM + 4.0 * OUT_DIM
+            sweep[str(e)] = {"us": us, "gbs_algorithmic": b / (us * 1e-6) / 1e9, "mean_used": Se,
+                             "vs_dense_roofline_measured": baselines["dense_roofline_us_measured_peak"] / us}
+
+    # end to end through the public API: pinned host v -> device, gemv, out -> pinned host
+    n_e2e = min(a.steps, 400)
+    hv = [torch.from_numpy(inputs.vector(IN_DIM, 7 + k, "t3")).pin_memory() for k in range(N_VECS)]
+    hout = torch.empty(OUT_DIM, dtype=torch.float32).pin_memory()
+    dv = torch.empty(IN_DIM, device=dev)
+    for k in range(20):
+        dv.copy_(hv[k % N_VECS], non_blocking=True)
+        mats[k % N_MATS].gemv(dv, EFFORT, out=outs[k % N_MATS])
+        hout.copy_(outs[k % N_MATS], non_blocking=True)
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for k in range(n_e2e):
+        dv.copy_(hv[k % N_VECS], non_blocking=True)
+        mats[k % N_MATS].gemv(dv, EFFORT, out=outs[k % N_MATS])
+        hout.copy_(outs[k % N_MATS], non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    barrier()
+    e2e_us = max_over_ranks(e0.elapsed_time(e1)) * 1000.0 / n_e2e / world
+
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        us_o, done, dt = time_oracle(2, 1, min_seconds=10.0)
+        cpu = cpu_baseline_record(us_o, done, dt)
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "us", "n_gpus": world, "steps": a.steps,
+                "warmup": a.warmup, "ms_per_step": us_per_step / 1000.0, "higher_is_better": False,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+                "config": workload_config(),
+                "gbs": alg_bytes / (us_per_step * 1e-6) / 1e9,
+                "roofline": roofline, "cpu_baseline": cpu,
+                "e2e": {"value": e2e_us, "unit": "us", "h2d_bytes_per_step": 4 * IN_DIM,
+                        "d2h_bytes_per_step": 4 * OUT_DIM},
+                "gpu_launches": 2 * a.steps, "clocks": clocks,
+                "phases_us": {"cutoff_dispatch": cut_us, "mac": mac_us},
+                "mean_used_products": S_mean, "baselines": baselines, "sweep": sweep}
+        print(json.dumps(line), flush=True)
+    for m in mats:
+        m.close()
+    ws.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

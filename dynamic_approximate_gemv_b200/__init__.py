@@ -54,6 +54,7 @@ def lib():
             "effort_prepare": [vp, i64, i64, f32, vp, ctypes.POINTER(vp)],
             "effort_gemv": [vp, vp, f32, vp, vp],
             "effort_gemv_ex": [vp, vp, ctypes.c_int, f32, vp, vp, vp, vp, vp],
+            "effort_gemv_split": [vp, vp, ctypes.c_int, f32, vp, vp, vp, vp, vp],
             "effort_check": [vp],
             "effort_workspace_create": [i64, i64, i32, ctypes.POINTER(vp)],
             "effort_workspace_destroy": [vp],
@@ -142,6 +143,19 @@ class PreparedMatrix:
                     raise ValueError(f"{nm} must be {dt} of shape {shp}")
         _check(lib().effort_gemv_ex(self._h, _ptr(v), _vdtype(v), ctypes.c_float(effort), _ptr(out), _ptr(cutoff),
                                     _ptr(count), _ptr(rowlen), _stream(v.device)), "effort_gemv")
+        return out
+
+    def gemv_split(self, v, effort, out, mid_event, stream=None):
+        """gemv that records `mid_event` (a recorded-once torch.cuda.Event) between the
+        cutoff/dispatch kernel and the multiply kernel, for per-phase timing."""
+        _need_cuda(v, "v")
+        _need_cuda(out, "out")
+        if not mid_event.cuda_event:
+            raise ValueError("mid_event has no CUDA event yet: record it once first")
+        st = stream if stream is not None else torch.cuda.current_stream(v.device)
+        _check(lib().effort_gemv_split(self._h, _ptr(v), _vdtype(v), ctypes.c_float(effort), _ptr(out), None, None,
+                                       ctypes.c_void_p(mid_event.cuda_event), ctypes.c_void_p(st.cuda_stream)),
+               "effort_gemv_split")
         return out
 
     def check(self):

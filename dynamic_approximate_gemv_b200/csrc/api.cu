@@ -17,11 +17,14 @@ cudaError_t launch_prep(const uint16_t* W, const HandleDesc* d_desc, int I, int 
                         cudaStream_t stream);
 cudaError_t launch_cutoff(const Jobs<1>& jobs, int I, int cl, cudaStream_t stream);
 cudaError_t launch_cutoff_batch(const Jobs<kMaxJobs>& jobs, int njobs, int I, int cl, cudaStream_t stream);
-cudaError_t launch_mac(const Jobs<1>& jobs, int T, int S, cudaStream_t stream);
-cudaError_t launch_mac_batch(const Jobs<kMaxJobs>& jobs, int njobs, int T, int S, cudaStream_t stream);
+cudaError_t launch_mac(const Jobs<1>& jobs, int P, int maxC, cudaStream_t stream);
+cudaError_t launch_mac_batch(const Jobs<kMaxJobs>& jobs, int njobs, int P, int maxC, cudaStream_t stream);
 cudaError_t launch_dense(const uint16_t* W, int I, int O, const void* v, int vdtype, float* out, float* part,
                          unsigned* tilecnt, int T, int S, cudaStream_t stream);
 int mac_ctas_per_sm();
+cudaError_t init_kernel_attributes();
+size_t cutoff_max_dynamic_smem();
+int cutoff_max_clusters(int cl, size_t smem);
 }  // namespace effort
 
 using namespace effort;
@@ -29,7 +32,12 @@ using namespace effort;
 namespace {
 
 struct Geometry {
-  int I, O, T, G, S, S_dense, cl;
+  int I, O, T, G;
+  int P;        // CTAs of the multiply kernel (stream-K over T * G units)
+  int maxC;     // most CTAs that share one output tile
+  int S_dense;  // row slices of the dense baseline
+  int cl;       // CTAs in the cutoff cluster
+  int dense_q16;  // dense-row threshold (share of the row surely used, x 65536)
 };
 
 struct WsBlock {
@@ -55,23 +63,39 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // Chooses the cutoff cluster size and the split-K slice counts.
 effort_status_t make_geometry(int64_t I, int64_t O, Geometry* g) {
   if (device_info() != cudaSuccess) return EFFORT_ERR_CUDA;
+  if (init_kernel_attributes() != cudaSuccess) return EFFORT_ERR_CUDA;
   g->I = (int)I;
   g->O = (int)O;
   g->T = (int)((O + kTW - 1) / kTW);
   g->G = (int)((I + kGroupRows - 1) / kGroupRows);
   g->cl = 0;
-  for (int cl : {8, 16}) {
-    if (cut_smem_bytes(g->I, cl) <= (size_t)g_smem_optin) {
+  const size_t dyn_max = cutoff_max_dynamic_smem();
+  for (int cl : {16, 8}) {  // the wider cluster halves each CTA's share of the rows
+    const size_t sm = cut_smem_bytes(g->I, cl);
+    if (sm <= dyn_max && cutoff_max_clusters(cl, sm) >= 1) {
       g->cl = cl;
       break;
     }
   }
   if (g->cl == 0) return EFFORT_ERR_UNSUPPORTED;
-  const int slots = g_num_sms * mac_ctas_per_sm();
-  int S = slots / g->T;
-  if (S < 1) S = 1;
-  if (S > g->G) S = g->G;
-  g->S = S;
+  const long long TU = (long long)g->T * g->G;
+  long long P = (long long)g_num_sms * mac_ctas_per_sm();
+  if (P > TU) P = TU;
+  g->P = (int)P;
+  int maxC = 1;
+  for (long long t = 0; t < g->T; ++t) {  // owner(u) = ((u + 1) * P - 1) / TU
+    const long long cf = ((t * g->G + 1) * P - 1) / TU, cl = (((t + 1) * g->G) * P - 1) / TU;
+    if (cl - cf + 1 > maxC) maxC = (int)(cl - cf + 1);
+  }
+  g->maxC = maxC;
+  // rows whose surely-used share reaches this fraction are read from the dense
+  // copy (2 B per weight, register accumulation) instead of their buckets
+  double frac = 0.5;
+  if (const char* env = getenv("EFFORT_DENSE_FRACTION")) {
+    const double f = atof(env);
+    if (f > 0.0 && f <= 1.0) frac = f;
+  }
+  g->dense_q16 = (int)(frac * 65536.0 + 0.5);
   int Sd = (g_num_sms * 8) / g->T;
   if (Sd < 1) Sd = 1;
   if (Sd > (int)((I + 7) / 8)) Sd = (int)((I + 7) / 8);
@@ -82,10 +106,11 @@ effort_status_t make_geometry(int64_t I, int64_t O, Geometry* g) {
 
 // One contiguous device block of scratch for `npairs` jobs.
 effort_status_t alloc_ws(const Geometry& g, int npairs, WsBlock* out, WsPtrs* slots) {
-  const int S = g.S > g.S_dense ? g.S : g.S_dense;
+  const int S = g.maxC > g.S_dense ? g.maxC : g.S_dense;
   const size_t per = align_up(256, 256)                                  // c, count, done, status
                      + align_up((size_t)g.T * 4, 256)                    // tilecnt
                      + align_up((size_t)g.G * 4, 256)                    // gcnt
+                     + align_up((size_t)g.G * g.T * 32, 256)             // ut
                      + align_up((size_t)g.G * kRecPerGroup * 16, 256)    // rec
                      + align_up((size_t)S * g.T * kTW * 4, 256);         // part
   const size_t bytes = per * (size_t)npairs;
@@ -110,6 +135,8 @@ effort_status_t alloc_ws(const Geometry& g, int npairs, WsBlock* out, WsPtrs* sl
     b += align_up((size_t)g.T * 4, 256);
     w.gcnt = (unsigned int*)b;
     b += align_up((size_t)g.G * 4, 256);
+    w.ut = (unsigned char*)b;
+    b += align_up((size_t)g.G * g.T * 32, 256);
     w.rec = (uint4*)b;
     b += align_up((size_t)g.G * kRecPerGroup * 16, 256);
     w.part = (float*)b;
@@ -292,7 +319,7 @@ static effort_status_t fill_job(effort_handle_t h, const WsPtrs& ws, const void*
   if (!effort_ok(effort)) return EFFORT_ERR_ARG;
   const long long N = (long long)h->g.I * (long long)h->g.O;
   const unsigned long long K = target_count(effort, N);
-  j->hd = h->d_desc;
+  j->hd = h->hd;
   j->v = v;
   j->out = out;
   j->cutoff_out = cutoff_out;
@@ -302,6 +329,7 @@ static effort_status_t fill_job(effort_handle_t h, const WsPtrs& ws, const void*
   j->K = K;
   j->mode = (K >= h->hd.kept_total) ? kModeAll : (K == 0 ? kModeNone : kModeSelect);
   j->vdtype = (int)v_dtype;
+  j->dense_q16 = h->g.dense_q16;
   return EFFORT_OK;
 }
 
@@ -315,7 +343,26 @@ effort_status_t effort_gemv_ex(effort_handle_t h, const void* v, effort_dtype_t 
   cudaStream_t s = (cudaStream_t)stream;
   h->last_stream = s;
   cudaError_t e = launch_cutoff(jobs, h->g.I, h->g.cl, s);
-  if (e == cudaSuccess) e = launch_mac(jobs, h->g.T, h->g.S, s);
+  if (e == cudaSuccess) e = launch_mac(jobs, h->g.P, h->g.maxC, s);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return EFFORT_ERR_CUDA;
+  }
+  return EFFORT_OK;
+}
+
+effort_status_t effort_gemv_split(effort_handle_t h, const void* v, effort_dtype_t v_dtype, float effort, float* out,
+                                  float* cutoff_out, uint64_t* count_out, void* mid_event, void* stream) {
+  if (!h || !mid_event) return EFFORT_ERR_ARG;
+  Jobs<1> jobs;
+  effort_status_t st = fill_job(h, h->slot, v, v_dtype, effort, out, cutoff_out, count_out, nullptr, &jobs.j[0]);
+  if (st != EFFORT_OK) return st;
+  DeviceGuard guard(h->dev);
+  cudaStream_t s = (cudaStream_t)stream;
+  h->last_stream = s;
+  cudaError_t e = launch_cutoff(jobs, h->g.I, h->g.cl, s);
+  if (e == cudaSuccess) e = cudaEventRecord((cudaEvent_t)mid_event, s);
+  if (e == cudaSuccess) e = launch_mac(jobs, h->g.P, h->g.maxC, s);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return EFFORT_ERR_CUDA;
@@ -409,7 +456,7 @@ effort_status_t effort_gemv_batched(effort_workspace_t ws, const effort_handle_t
       if (st != EFFORT_OK) return st;
     }
     cudaError_t e = launch_cutoff_batch(jobs, nj, I, ws->g.cl, s);
-    if (e == cudaSuccess) e = launch_mac_batch(jobs, nj, ws->g.T, ws->g.S, s);
+    if (e == cudaSuccess) e = launch_mac_batch(jobs, nj, ws->g.P, ws->g.maxC, s);
     if (e != cudaSuccess) {
       cudaGetLastError();
       return EFFORT_ERR_CUDA;

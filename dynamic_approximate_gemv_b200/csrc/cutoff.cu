@@ -8,18 +8,24 @@
 //   chart   x_ik = fl32(|v_i| * p_ik), kept in shared memory as fp32 bit
 //           patterns (non-negative floats order like their bit patterns).
 //   topK    c = max{x : sum of probe weights of chart entries >= x is >= K}.
-//           Weighted radix select over the bit patterns, 3 passes of
-//           12 / 10 / 9 bits; each pass builds CTA-local weighted histograms,
-//           merges them across the cluster through distributed shared memory
-//           (each CTA sums one slice of bins and broadcasts it), and picks the
-//           digit where the weight counted from the top first reaches K.
+//           Weighted radix select over the bit patterns.  The first digit
+//           (bits 30..19) is chosen cluster-wide: CTA-local weighted
+//           histograms are summed by every CTA through distributed shared
+//           memory.  Each CTA then lists its chart entries that fall in the
+//           chosen bin, every CTA gathers all lists and finishes the select
+//           locally (bits 18..9, then 8..0); all CTAs reach the same c.  If the
+//           bin holds too many entries, the last two digits are also chosen
+//           cluster-wide.
 //   dispatch per row: the probes that pass c narrow the rank range of the
 //           row's selection boundary; the checkpoint magnitudes inside that
 //           range give k_i, the number of checkpoint blocks of H ranks that are
-//           used entirely.  Rows with 2 * k_i * H >= n are "dense" (read from
-//           the dense copy), other active rows are "sparse" (read from the
-//           sorted buckets), rows whose largest product is below c are off.
-//           Records go to fixed slots of their 32-row group.
+//           used entirely.  The row's exact fp16 threshold tau_i (smallest
+//           magnitude whose product with |v_i| reaches c) turns the product
+//           rule into a magnitude compare.  Rows with k_i * H >= f * n (f the
+//           dense fraction, 1/2 by default) are "dense" (read from the dense
+//           copy), other active rows are "sparse" (read from the sorted
+//           buckets), rows whose largest product is below c are off.  Records
+//           {row, v_i, tau_i, k_i} go to fixed slots of their 32-row group.
 #include <cooperative_groups.h>
 
 #include "effort_internal.cuh"
@@ -28,10 +34,14 @@ namespace cg = cooperative_groups;
 
 namespace effort {
 
-__device__ __forceinline__ float load_v(const Job& jb, int i) {
-  if (jb.vdtype == 1) return __half2float(reinterpret_cast<const __half*>(jb.v)[i]);
-  return reinterpret_cast<const float*>(jb.v)[i];
-}
+struct CutShared {
+  unsigned warp_tot[32];
+  unsigned sel_digit;
+  unsigned sel_krem;
+  unsigned ncand;       // this CTA's entries in the first-pass bin
+  unsigned cand_off[17];
+  unsigned cand_total;
+};
 
 // Inclusive prefix sum over the block (blockDim.x == kCutThreads).
 __device__ __forceinline__ unsigned block_inclusive_scan(unsigned x, unsigned* warp_tot, unsigned& total) {
@@ -59,23 +69,45 @@ __device__ __forceinline__ unsigned block_inclusive_scan(unsigned x, unsigned* w
   return x + before;
 }
 
-struct CutShared {
-  unsigned warp_tot[32];
-  unsigned sel_digit;
-  unsigned sel_krem;
-};
-
-// One radix pass over `bits` bits starting at `shift`.
+// Over a complete histogram of B digits: D = max{d : weight of digits >= d
+// reaches krem}; also the weight still needed inside digit D.
 template <int B>
-__device__ void radix_pass(cg::cluster_group& cluster, int cl, int crank, int shift, const unsigned* chart,
-                           int nelem, const int* pw, unsigned* lh, unsigned* mg, unsigned& prefix,
-                           unsigned& pmask, unsigned& krem, CutShared& cs) {
+__device__ void find_crossing(const unsigned* hist, unsigned krem, CutShared& cs, unsigned& digit, unsigned& knew) {
+  constexpr int q = (B + kCutThreads - 1) / kCutThreads;
+  const int lo = threadIdx.x * q, hi = min(B, lo + q);
+  unsigned local = 0;
+  for (int b = lo; b < hi; ++b) local += hist[b];
+  unsigned total;
+  const unsigned incl = block_inclusive_scan(local, cs.warp_tot, total);
+  unsigned cum = total - incl;  // weight of all digits above my range
+  for (int b = hi - 1; b >= lo; --b) {
+    const unsigned nb = hist[b];
+    if (cum < krem && cum + nb >= krem) {
+      cs.sel_digit = (unsigned)b;
+      cs.sel_krem = krem - cum;
+    }
+    cum += nb;
+  }
+  __syncthreads();
+  digit = cs.sel_digit;
+  knew = cs.sel_krem;
+  __syncthreads();
+}
+
+// Cluster-wide radix pass (used when the first-pass bin is crowded).
+template <int B>
+__device__ void cluster_radix_pass(cg::cluster_group& cluster, int cl, int crank, int shift, const unsigned* chart,
+                                   int RP, int nr, const int* pw, unsigned* lh, unsigned* mg, unsigned& prefix,
+                                   unsigned& pmask, unsigned& krem, CutShared& cs) {
   for (int b = threadIdx.x; b < B; b += blockDim.x) lh[b] = 0u;
   __syncthreads();
-  for (int e = threadIdx.x; e < nelem; e += blockDim.x) {
-    const unsigned x = chart[e];
-    const int w = pw[e & (kP - 1)];
-    if (w > 0 && (x & pmask) == prefix) atomicAdd(&lh[(x >> shift) & (B - 1)], (unsigned)w);
+  for (int k = 0; k < kP; ++k) {
+    const int w = pw[k];
+    if (w == 0) continue;
+    for (int r = threadIdx.x; r < nr; r += blockDim.x) {
+      const unsigned x = chart[(size_t)k * RP + r];
+      if ((x & pmask) == prefix) atomicAdd(&lh[(x >> shift) & (B - 1)], (unsigned)w);
+    }
   }
   __syncthreads();
   cluster.sync();
@@ -87,27 +119,29 @@ __device__ void radix_pass(cg::cluster_group& cluster, int cl, int crank, int sh
     for (int r = 0; r < cl; ++r) cluster.map_shared_rank(mg, r)[bin] = s;
   }
   cluster.sync();
-  // D = max{digit d : weight of digits >= d reaches krem}
-  constexpr int q = (B + kCutThreads - 1) / kCutThreads;
-  const int lo = threadIdx.x * q, hi = min(B, lo + q);
-  unsigned local = 0;
-  for (int b = lo; b < hi; ++b) local += mg[b];
-  unsigned total;
-  const unsigned incl = block_inclusive_scan(local, cs.warp_tot, total);
-  unsigned cum = total - incl;  // weight of all digits above my range
-  for (int b = hi - 1; b >= lo; --b) {
-    const unsigned nb = mg[b];
-    if (cum < krem && cum + nb >= krem) {
-      cs.sel_digit = (unsigned)b;
-      cs.sel_krem = krem - cum;
-    }
-    cum += nb;
+  unsigned digit, knew;
+  find_crossing<B>(mg, krem, cs, digit, knew);
+  prefix |= digit << shift;
+  pmask |= (unsigned)(B - 1) << shift;
+  krem = knew;
+}
+
+// Local radix pass over gathered (value, weight) candidates.
+template <int B>
+__device__ void local_radix_pass(int shift, const unsigned* val, const unsigned short* wt, int n, unsigned* hist,
+                                 unsigned& prefix, unsigned& pmask, unsigned& krem, CutShared& cs) {
+  for (int b = threadIdx.x; b < B; b += blockDim.x) hist[b] = 0u;
+  __syncthreads();
+  for (int e = threadIdx.x; e < n; e += blockDim.x) {
+    const unsigned x = val[e];
+    if ((x & pmask) == prefix) atomicAdd(&hist[(x >> shift) & (B - 1)], (unsigned)wt[e]);
   }
   __syncthreads();
-  prefix |= cs.sel_digit << shift;
+  unsigned digit, knew;
+  find_crossing<B>(hist, krem, cs, digit, knew);
+  prefix |= digit << shift;
   pmask |= (unsigned)(B - 1) << shift;
-  krem = cs.sel_krem;
-  __syncthreads();
+  krem = knew;
 }
 
 template <int NJ>
@@ -118,53 +152,186 @@ __global__ void __launch_bounds__(kCutThreads, 1) k_cutoff_dispatch(const __grid
   cg::cluster_group cluster = cg::this_cluster();
   const int crank = (int)cluster.block_rank();
   const Job& jb = jobs.j[blockIdx.x / cl];
-
-  __shared__ HandleDesc d;
   __shared__ CutShared cs;
-  if (threadIdx.x < (int)(sizeof(HandleDesc) / 4))
-    reinterpret_cast<int*>(&d)[threadIdx.x] = reinterpret_cast<const int*>(jb.hd)[threadIdx.x];
-  __syncthreads();
-
-  const int I = d.I, n = d.n, C = d.C, H = d.H;
+  __shared__ int s_prank[kP], s_pw[kP];
+  // every field used below is read once from the parameter bank into registers
+  const int I = jb.hd.I, n = jb.hd.n, C = jb.hd.C, H = jb.hd.H;
+  const uint16_t* __restrict__ ckmag = jb.hd.ckmag;
+  const uint16_t* __restrict__ probes = jb.hd.probes;
+  const void* vptr = jb.v;
+  const int vdtype = jb.vdtype, dense_q16 = jb.dense_q16;
+  unsigned* __restrict__ status = jb.ws.status;
+  uint4* __restrict__ rec = jb.ws.rec;
+  unsigned* __restrict__ gcnt = jb.ws.gcnt;
+  unsigned char* __restrict__ ut = jb.ws.ut;
+  const uint8_t* __restrict__ cntt = jb.hd.cnt;
+  const int T = jb.hd.T;
+  unsigned* __restrict__ rowlen_out = jb.rowlen_out;
+  const unsigned Kt = (unsigned)jb.K;
+  if (threadIdx.x < kP) {
+    s_prank[threadIdx.x] = jb.hd.prank[threadIdx.x];
+    s_pw[threadIdx.x] = jb.hd.pw[threadIdx.x];
+  }
   const int RP = cut_rows_per_cta(I, cl);
   const int i0 = crank * RP;
   const int nr = max(0, min(I, i0 + RP) - i0);
   const int G = (I + kGroupRows - 1) / kGroupRows;
 
-  extern __shared__ unsigned smem[];
-  unsigned* chart = smem;
-  float* vs = reinterpret_cast<float*>(chart + (size_t)RP * kP);
-  unsigned* h0 = reinterpret_cast<unsigned*>(vs + RP);
-  unsigned* m0 = h0 + kBins0;
-  unsigned* h1 = m0 + kBins0;
+  extern __shared__ __align__(16) unsigned smem[];
+  unsigned* chart = smem;                                                    // [kP][RP], column k at k * RP
+  float* vs = reinterpret_cast<float*>(chart + (size_t)RP * kP);             // RP
+  unsigned* h0 = reinterpret_cast<unsigned*>(vs + RP);                       // kBins0
+  unsigned* cval = h0 + kBins0;                                              // kCandLocal
+  unsigned short* cwt = reinterpret_cast<unsigned short*>(cval + kCandLocal);  // kCandLocal
+  unsigned* uni = reinterpret_cast<unsigned*>(cwt + kCandLocal);             // shared area
+  unsigned* mg0 = uni;                                                       // merged first-pass histogram
+  unsigned* gval = uni;                                                      // gathered candidates
+  unsigned short* gwt = reinterpret_cast<unsigned short*>(uni + kCandTotal);
+  unsigned* h1 = uni;                                                        // fallback passes
   unsigned* m1 = h1 + kBins1;
   unsigned* h2 = m1 + kBins1;
   unsigned* m2 = h2 + kBins2;
 
   int mode = jb.mode;
+  if (threadIdx.x == 0) cs.ncand = 0u;
+  // ---- v and probes (one thread per row), and an L2 prefetch of the row's
+  // checkpoint magnitudes for the dispatch
   bool bad = false;
   for (int r = threadIdx.x; r < nr; r += blockDim.x) {
-    const float x = load_v(jb, i0 + r);
+    const int i = i0 + r;
+    uint4 p0 = make_uint4(0, 0, 0, 0), p1 = p0;
+    if (mode == kModeSelect) {
+      p0 = reinterpret_cast<const uint4*>(probes + (size_t)i * kP)[0];
+      p1 = reinterpret_cast<const uint4*>(probes + (size_t)i * kP)[1];
+    }
+    const float x = (vdtype == 1) ? __half2float(reinterpret_cast<const __half*>(vptr)[i])
+                                  : reinterpret_cast<const float*>(vptr)[i];
+    const char* ck = reinterpret_cast<const char*>(ckmag + (size_t)i * (C + 1));
+    for (int b = 0; b < (C + 1) * 2; b += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(ck + b));
     if (!isfinite(x)) bad = true;
     vs[r] = x;
-  }
-  if (bad) atomicOr(jb.ws.status, kStatusNonfiniteV);
-  __syncthreads();
-  if (mode == kModeSelect) {
-    for (int e = threadIdx.x; e < nr * kP; e += blockDim.x) {
-      const int r = e >> 4, k = e & (kP - 1);
-      const float p = __half2float(__ushort_as_half(d.probes[(size_t)(i0 + r) * kP + k]));
-      chart[e] = __float_as_uint(__fmul_rn(fabsf(vs[r]), p));
+    if (mode == kModeSelect) {
+      const float av = fabsf(x);
+      const unsigned short* ph0 = reinterpret_cast<const unsigned short*>(&p0);
+      const unsigned short* ph1 = reinterpret_cast<const unsigned short*>(&p1);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        chart[(size_t)k * RP + r] = __float_as_uint(__fmul_rn(av, __half2float(__ushort_as_half(ph0[k]))));
+        chart[(size_t)(8 + k) * RP + r] = __float_as_uint(__fmul_rn(av, __half2float(__ushort_as_half(ph1[k]))));
+      }
     }
   }
+  if (bad) atomicOr(status, kStatusNonfiniteV);
   __syncthreads();
 
   unsigned prefix = 0u, pmask = 0u;
-  unsigned krem = (unsigned)jb.K;
+  unsigned krem = Kt;
+  bool split_exit = false;  // cluster barrier arrived early, to be waited on at exit
   if (mode == kModeSelect) {
-    radix_pass<kBins0>(cluster, cl, crank, 19, chart, nr * kP, d.pw, h0, m0, prefix, pmask, krem, cs);
-    radix_pass<kBins1>(cluster, cl, crank, 9, chart, nr * kP, d.pw, h1, m1, prefix, pmask, krem, cs);
-    radix_pass<kBins2>(cluster, cl, crank, 0, chart, nr * kP, d.pw, h2, m2, prefix, pmask, krem, cs);
+    // ---- first digit, cluster-wide.  Local weighted histogram; its nonzero
+    // bins are added into the owner CTA's slice (bin / (kBins0 / cl)) with
+    // distributed shared memory atomics; after one cluster barrier every CTA
+    // reads the whole merged histogram.
+    const int per = kBins0 / cl;
+    unsigned* own = mg0;  // this CTA's merged slice lives at the start of the shared area
+    for (int b = threadIdx.x; b < kBins0; b += blockDim.x) h0[b] = 0u;
+    for (int b = threadIdx.x; b < per; b += blockDim.x) own[b] = 0u;
+    __syncthreads();
+    for (int e = threadIdx.x; e < nr * kP; e += blockDim.x) {
+      const int k = e / nr, r = e - k * nr;
+      const int wk = s_pw[k];
+      if (wk > 0) atomicAdd(&h0[(chart[(size_t)k * RP + r] >> 19) & (kBins0 - 1)], (unsigned)wk);
+    }
+    cluster.sync();  // every CTA's slice is zeroed and its local histogram complete
+    for (int b = threadIdx.x; b < kBins0; b += blockDim.x) {
+      const unsigned x = h0[b];
+      if (x) atomicAdd(cluster.map_shared_rank(own, b / per) + (b % per), x);
+    }
+    cluster.sync();  // merged slices complete
+    {
+      unsigned* full = h0;  // the local histogram is no longer needed: reuse it for the merged copy
+      constexpr int kPerThread = kBins0 / kCutThreads;
+      unsigned x[kPerThread];
+#pragma unroll
+      for (int u = 0; u < kPerThread; ++u) {
+        const int b = threadIdx.x + u * kCutThreads;
+        x[u] = *(cluster.map_shared_rank(own, b / per) + (b % per));
+      }
+      __syncthreads();
+#pragma unroll
+      for (int u = 0; u < kPerThread; ++u) full[threadIdx.x + u * kCutThreads] = x[u];
+      __syncthreads();
+    }
+    unsigned digit, knew;
+    find_crossing<kBins0>(h0, Kt, cs, digit, knew);
+    prefix = digit << 19;
+    pmask = (unsigned)(kBins0 - 1) << 19;
+    krem = knew;
+    // ---- this CTA's entries in the chosen bin
+    for (int e = threadIdx.x; e < nr * kP; e += blockDim.x) {
+      const int k = e / nr, r = e - k * nr;
+      const int wk = s_pw[k];
+      const unsigned x = chart[(size_t)k * RP + r];
+      if (wk > 0 && (x & pmask) == prefix) {
+        const unsigned slot = atomicAdd(&cs.ncand, 1u);
+        if (slot < (unsigned)kCandLocal) {
+          cval[slot] = x;
+          cwt[slot] = (unsigned short)wk;
+        }
+      }
+    }
+    __syncthreads();
+    cluster.sync();  // every list complete; no CTA reads another's merged slice any more
+    if (threadIdx.x == 0) {
+      unsigned tot = 0;
+      bool over = false;
+      for (int r = 0; r < cl; ++r) {
+        const unsigned nc = *cluster.map_shared_rank(&cs.ncand, r);
+        over |= nc > (unsigned)kCandLocal;
+        cs.cand_off[r] = tot;
+        tot += nc;
+      }
+      cs.cand_off[cl] = tot;
+      cs.cand_total = over ? 0xFFFFFFFFu : tot;
+    }
+    __syncthreads();
+    const unsigned total = cs.cand_total;
+    if (total <= (unsigned)kCandTotal) {
+      // gather every CTA's list and finish locally (same multiset, same c everywhere)
+      for (unsigned q0 = 0; q0 < total; q0 += 4u * kCutThreads) {
+        unsigned v4[4];
+        unsigned short w4[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {  // issue the remote loads of four candidates together
+          const unsigned q = q0 + threadIdx.x + (unsigned)u * kCutThreads;
+          v4[u] = 0u;
+          w4[u] = 0;
+          if (q < total) {
+            int r = 0;
+            while (q >= cs.cand_off[r + 1]) ++r;
+            const unsigned k = q - cs.cand_off[r];
+            v4[u] = cluster.map_shared_rank(cval, r)[k];
+            w4[u] = cluster.map_shared_rank(cwt, r)[k];
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const unsigned q = q0 + threadIdx.x + (unsigned)u * kCutThreads;
+          if (q < total) {
+            gval[q] = v4[u];
+            gwt[q] = w4[u];
+          }
+        }
+      }
+      asm volatile("barrier.cluster.arrive.release.aligned;\n" ::: "memory");
+      split_exit = true;
+      __syncthreads();
+      local_radix_pass<kBins1>(9, gval, gwt, (int)total, h0, prefix, pmask, krem, cs);
+      local_radix_pass<kBins2>(0, gval, gwt, (int)total, h0, prefix, pmask, krem, cs);
+    } else {
+      cluster_radix_pass<kBins1>(cluster, cl, crank, 9, chart, RP, nr, s_pw, h1, m1, prefix, pmask, krem, cs);
+      cluster_radix_pass<kBins2>(cluster, cl, crank, 0, chart, RP, nr, s_pw, h2, m2, prefix, pmask, krem, cs);
+    }
   }
   const float c = (mode == kModeAll) ? 0.0f : (mode == kModeNone) ? __int_as_float(0x7F800000) : __uint_as_float(prefix);
   const unsigned cbits = __float_as_uint(c);
@@ -176,42 +343,74 @@ __global__ void __launch_bounds__(kCutThreads, 1) k_cutoff_dispatch(const __grid
     if (jb.cutoff_out) jb.cutoff_out[0] = c;
   }
 
-  // dispatch: one thread per row; a warp covers one 32-row group
+  // ---- dispatch: one thread per row; a warp covers one 32-row group
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int base = 0; base < RP; base += blockDim.x) {
     const int r = base + threadIdx.x;
     const int i = i0 + r;
     const bool valid = r < nr;
     int cls = kClassOff, ki = 0;
+    unsigned tau = 0x7C00u;
     float vi = 0.0f;
     if (valid) {
       vi = vs[r];
       if (mode == kModeAll) {
         cls = kClassDense;
         ki = C;
+        tau = 0u;
       } else if (mode == kModeSelect) {
         const float av = fabsf(vi);
+        // tau: the smallest fp16 magnitude m with fl32(|v_i| * m) >= c (0x7C00 if
+        // none); fl32(|v_i| * m) is non-decreasing in m, so |w| >= tau <=> used.
+        // Start from the fp16 rounding of c / |v_i| and settle it with exact
+        // product tests; a bisection over all magnitudes covers the rest.
+        const float q = c * (1.0f / av);  // inf when av == 0
+        unsigned lo = 0u, hi = 0x7C00u;
+        if (q < 65504.0f) {
+          const unsigned g = (unsigned)__half_as_ushort(__float2half_rd(q)) & 0x7FFFu;
+          const unsigned a = g > 2u ? g - 2u : 0u, b = min(g + 3u, 0x7C00u);
+          // [a, b) brackets the answer when the guess is within two ulps
+          const bool a_fails = (a == 0u) || (__fmul_rn(av, __half2float(__ushort_as_half((unsigned short)(a - 1u)))) < c);
+          const bool b_passes = (b == 0x7C00u) || (__fmul_rn(av, __half2float(__ushort_as_half((unsigned short)b))) >= c);
+          if (a_fails && b_passes) {
+            lo = a;
+            hi = b;
+          }
+        }
+        while (lo < hi) {
+          const unsigned mid = (lo + hi) >> 1;
+          if (__fmul_rn(av, __half2float(__ushort_as_half((unsigned short)mid))) >= c) hi = mid;
+          else lo = mid + 1u;
+        }
+        tau = lo;
+        // probes narrow the rank range of the row's boundary
         int last_sel = -1, first_unsel = n;
         for (int k = 0; k < kP; ++k) {
-          const int rk = d.prank[k];
+          const int rk = s_prank[k];
           if (rk < 0) continue;
-          if (chart[r * kP + k] >= cbits) last_sel = rk;
+          if (chart[(size_t)k * RP + r] >= cbits) last_sel = rk;
           else if (first_unsel == n) first_unsel = rk;
         }
         const int known = min(C, (last_sel + 1) / H);
         const int kend = (first_unsel >= n) ? C : min(C - 1, (first_unsel + 1 + H - 1) / H - 1);
         ki = known;
-        const uint16_t* ck = d.ckmag + (size_t)i * (C + 1);
-        for (int k = known; k < kend; ++k) {
-          const float m = __half2float(__ushort_as_half(ck[1 + k]));
-          if (__fmul_rn(av, m) >= c) ki = k + 1;
-          else break;
+        const uint16_t* ck = ckmag + (size_t)i * (C + 1);
+        // checkpoints in the window, loaded together; the used ones lead the window
+        for (int k0 = known; k0 < kend; k0 += 16) {
+          unsigned short m[16];
+#pragma unroll
+          for (int u = 0; u < 16; ++u) m[u] = (k0 + u < kend) ? ck[1 + k0 + u] : (unsigned short)0;
+          int cnt = 0;
+#pragma unroll
+          for (int u = 0; u < 16; ++u) cnt += (k0 + u < kend && (unsigned)m[u] >= tau) ? 1 : 0;
+          ki += cnt;
+          if (cnt < 16) break;
         }
-        bool active = (ki > 0) || (last_sel >= 0);
-        if (!active) active = __fmul_rn(av, __half2float(__ushort_as_half(ck[0]))) >= c;
-        if (active) cls = (2 * ki * H >= n) ? kClassDense : kClassSparse;
+        const bool active = (ki > 0) || (last_sel >= 0) || ((unsigned)ck[0] >= tau);
+        if (active)
+          cls = ((long long)ki * H * 65536 >= (long long)n * dense_q16) ? kClassDense : kClassSparse;
       }
-      if (jb.rowlen_out) jb.rowlen_out[i] = (mode == kModeAll) ? (unsigned)n : 0u;
+      if (rowlen_out) rowlen_out[i] = (mode == kModeAll) ? (unsigned)n : 0u;
     }
     const unsigned bs = __ballot_sync(0xFFFFFFFFu, cls == kClassSparse);
     const unsigned bd = __ballot_sync(0xFFFFFFFFu, cls == kClassDense);
@@ -219,23 +418,76 @@ __global__ void __launch_bounds__(kCutThreads, 1) k_cutoff_dispatch(const __grid
     // a group is written only by the CTA whose row range holds it
     if (base + warp * kGroupRows < RP && g < G) {
       const unsigned lt = (1u << lane) - 1u;
-      const uint4 rec = make_uint4((unsigned)i, __float_as_uint(vi), (unsigned)ki, (unsigned)cls);
-      if (cls == kClassSparse) jb.ws.rec[(size_t)g * kRecPerGroup + __popc(bs & lt)] = rec;
-      if (cls == kClassDense) jb.ws.rec[(size_t)g * kRecPerGroup + 32 + __popc(bd & lt)] = rec;
-      if (lane == 0) jb.ws.gcnt[g] = (unsigned)__popc(bs) | ((unsigned)__popc(bd) << 8);
+      const uint4 r4 = make_uint4((unsigned)i, __float_as_uint(vi), tau, (unsigned)ki);
+      if (cls == kClassSparse) {
+        const int p = __popc(bs & lt);
+        rec[(size_t)g * kRecPerGroup + p] = r4;
+        // the read bound of this row in every tile: entries of the tile among the
+        // first min((k+1) H, n) ranks (255 saturates: read the whole bucket)
+        const uint8_t* crow = cntt + ((size_t)i * C + min(ki, C - 1)) * T;
+        unsigned char* urow = ut + (size_t)g * T * 32 + p;
+        for (int t = 0; t < T; ++t) urow[(size_t)t * 32] = crow[t];
+      }
+      if (cls == kClassDense) rec[(size_t)g * kRecPerGroup + 32 + __popc(bd & lt)] = r4;
+      if (lane == 0) gcnt[g] = (unsigned)__popc(bs) | ((unsigned)__popc(bd) << 8);
     }
   }
+  // other CTAs may still be reading this CTA's candidate list
+  if (split_exit) asm volatile("barrier.cluster.wait.acquire.aligned;\n" ::: "memory");
+}
+
+// Largest dynamic shared memory a cutoff CTA may use on this device: the
+// opt-in limit minus the kernel's static shared memory.
+size_t cutoff_max_dynamic_smem() {
+  int dev = 0, optin = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return 0;
+  cudaFuncAttributes fa1, fa16;
+  if (cudaFuncGetAttributes(&fa1, k_cutoff_dispatch<1>) != cudaSuccess) return 0;
+  if (cudaFuncGetAttributes(&fa16, k_cutoff_dispatch<kMaxJobs>) != cudaSuccess) return 0;
+  const size_t st = fa1.sharedSizeBytes > fa16.sharedSizeBytes ? fa1.sharedSizeBytes : fa16.sharedSizeBytes;
+  return (size_t)optin > st ? (size_t)optin - st : 0;
+}
+
+// Kernel attributes are set once per device (outside any stream capture):
+// the largest dynamic shared memory the chart may need and 16-CTA clusters.
+cudaError_t cutoff_attributes() {
+  const int dyn = (int)cutoff_max_dynamic_smem();
+  if (dyn <= 0) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(k_cutoff_dispatch<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k_cutoff_dispatch<kMaxJobs>, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_cutoff_dispatch<1>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k_cutoff_dispatch<kMaxJobs>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  return e;
+}
+
+// How many clusters of `cl` CTAs with `smem` bytes each the device can hold
+// at once (0: this cluster shape cannot be launched here).
+int cutoff_max_clusters(int cl, size_t smem) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)cl, 1, 1);
+  cfg.blockDim = dim3(kCutThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)cl;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, k_cutoff_dispatch<1>, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n;
 }
 
 template <int NJ>
 cudaError_t launch_cutoff_t(const Jobs<NJ>& jobs, int njobs, int I, int cl, cudaStream_t stream) {
   const size_t smem = cut_smem_bytes(I, cl);
-  cudaError_t e = cudaFuncSetAttribute(k_cutoff_dispatch<NJ>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  if (cl > 8) {
-    e = cudaFuncSetAttribute(k_cutoff_dispatch<NJ>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    if (e != cudaSuccess) return e;
-  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(cl * njobs), 1, 1);
   cfg.blockDim = dim3(kCutThreads, 1, 1);

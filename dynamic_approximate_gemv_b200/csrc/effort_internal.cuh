@@ -26,7 +26,7 @@ constexpr int kTW = 256;         // output-tile width (u8 local column)
 constexpr int kCap = 256;        // bucket capacity (entries)
 constexpr int kP = 16;           // probes per row
 constexpr int kCutThreads = 1024;
-constexpr int kMacThreads = 256;
+constexpr int kMacThreads = 512;
 constexpr int kMacWarps = kMacThreads / 32;
 constexpr int kPrepThreads = 1024;
 constexpr int kDenseThreads = 256;
@@ -62,14 +62,15 @@ struct WsPtrs {
   unsigned long long* count;    // running |S|
   unsigned int* done;           // CTAs of the multiply kernel that finished
   unsigned int* tilecnt;        // [T] split-K arrivals per tile
-  uint4* rec;                   // [G][64] dispatch records {row, v bits, k, class}
+  uint4* rec;                   // [G][64] dispatch records {row, v bits, tau (fp16 bits), k}
   unsigned int* gcnt;           // [G] (#sparse) | (#dense << 8)
-  float* part;                  // [S][T * 256] split-K partial sums
+  unsigned char* ut;            // [G][T][32]: read bound U of sparse slot p of group g in tile t
+  float* part;                  // per-tile partial sums of the CTAs that share a tile
   unsigned int* status;         // sticky device status bits
 };
 
 struct Job {
-  const HandleDesc* hd;
+  HandleDesc hd;  // by value: kernels read it from the parameter bank
   const void* v;
   float* out;
   float* cutoff_out;
@@ -78,7 +79,9 @@ struct Job {
   WsPtrs ws;
   unsigned long long K;
   int mode;
-  int vdtype;  // 0 f32, 1 f16
+  int vdtype;     // 0 f32, 1 f16
+  int dense_q16;  // a row is read densely once this share (x 65536) of it is surely used
+  int pad0;
 };
 
 template <int NJ>
@@ -93,9 +96,21 @@ __host__ __device__ inline int cut_rows_per_cta(int I, int cl) {
 }
 // radix-select digits: bits [30:19], [18:9], [8:0] of the non-negative fp32 chart
 constexpr int kBins0 = 4096, kBins1 = 1024, kBins2 = 512;
+constexpr int kCandLocal = 2048;  // crossing-bin candidates one cutoff CTA can hold
+constexpr int kCandTotal = 4096;  // candidates gathered from the whole cluster
+// dynamic shared memory of a cutoff CTA: chart, v, the first-pass histogram,
+// its candidate list, and one area shared by the merged histogram, the
+// gathered candidates and the fallback passes
+__host__ __device__ inline size_t cut_union_bytes() {
+  const size_t merged = (size_t)kBins0 * 4;
+  const size_t gathered = (size_t)kCandTotal * 6;
+  const size_t fallback = 2 * (size_t)(kBins1 + kBins2) * 4;
+  size_t m = merged > gathered ? merged : gathered;
+  return m > fallback ? m : fallback;
+}
 __host__ __device__ inline size_t cut_smem_bytes(int I, int cl) {
-  size_t rp = (size_t)cut_rows_per_cta(I, cl);
-  return rp * kP * 4 + rp * 4 + 2 * (size_t)(kBins0 + kBins1 + kBins2) * 4 + 64;
+  const size_t rp = (size_t)cut_rows_per_cta(I, cl);
+  return rp * kP * 4 + rp * 4 + (size_t)kBins0 * 4 + (size_t)kCandLocal * 6 + cut_union_bytes() + 64;
 }
 
 }  // namespace effort

@@ -18,6 +18,8 @@
 //      checkpoint.
 #include "effort_internal.cuh"
 
+#define EFFORT_PREP_SMEM_MAX (32768 * 4)  // keys of the widest supported row
+
 namespace effort {
 
 __device__ __forceinline__ void bitonic_sort_u32(uint32_t* s, int Np) {
@@ -104,14 +106,16 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
   }
 }
 
+cudaError_t prep_attributes() {
+  return cudaFuncSetAttribute(k_prep_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, EFFORT_PREP_SMEM_MAX);
+}
+
 cudaError_t launch_prep(const uint16_t* W, const HandleDesc* d_desc, int I, int O, uint16_t* vals, uint8_t* idx,
                         uint16_t* wdense, uint16_t* probes, uint16_t* ckmag, uint8_t* cnt, unsigned int* status,
                         cudaStream_t stream) {
   int Np = 1;
   while (Np < O) Np <<= 1;
   const size_t smem = (size_t)Np * 4;
-  cudaError_t e = cudaFuncSetAttribute(k_prep_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
   k_prep_rows<<<I, kPrepThreads, smem, stream>>>(W, d_desc, Np, vals, idx, wdense, probes, ckmag, cnt, status);
   return cudaGetLastError();
 }

@@ -103,6 +103,17 @@ effort_status_t effort_gemv_ex(effort_handle_t h, const void* v, effort_dtype_t 
                                void* stream);
 
 /*
+ * effort_gemv_split -- effort_gemv_ex that also records `mid_event` (a
+ *   cudaEvent_t passed as void*, created by the caller) on the stream between
+ *   the cutoff/dispatch kernel and the multiply kernel, so that each phase can
+ *   be timed with events.  The multiply kernel then starts after the event
+ *   instead of launching early against the first kernel.  mid_event non-NULL.
+ */
+effort_status_t effort_gemv_split(effort_handle_t h, const void* v, effort_dtype_t v_dtype, float effort,
+                                  float* out, float* cutoff_out, uint64_t* count_out, void* mid_event,
+                                  void* stream);
+
+/*
  * effort_check -- synchronises the handle's last stream and reports whether a
  *   call since the previous check saw a non-finite entry of v
  *   (EFFORT_ERR_NONFINITE; those calls' outputs are unspecified) or an internal
