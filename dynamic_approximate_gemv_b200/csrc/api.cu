@@ -17,8 +17,8 @@ cudaError_t launch_prep(const uint16_t* W, const HandleDesc* d_desc, int I, int 
                         cudaStream_t stream);
 cudaError_t launch_cutoff(const Jobs<1>& jobs, int I, int cl, cudaStream_t stream);
 cudaError_t launch_cutoff_batch(const Jobs<kMaxJobs>& jobs, int njobs, int I, int cl, cudaStream_t stream);
-cudaError_t launch_mac(const Jobs<1>& jobs, int P, int maxC, cudaStream_t stream);
-cudaError_t launch_mac_batch(const Jobs<kMaxJobs>& jobs, int njobs, int P, int maxC, cudaStream_t stream);
+cudaError_t launch_mac(const Jobs<1>& jobs, int T, int S, cudaStream_t stream);
+cudaError_t launch_mac_batch(const Jobs<kMaxJobs>& jobs, int njobs, int T, int S, cudaStream_t stream);
 cudaError_t launch_dense(const uint16_t* W, int I, int O, const void* v, int vdtype, float* out, float* part,
                          unsigned* tilecnt, int T, int S, cudaStream_t stream);
 int mac_ctas_per_sm();
@@ -33,8 +33,7 @@ namespace {
 
 struct Geometry {
   int I, O, T, G;
-  int P;        // CTAs of the multiply kernel (stream-K over T * G units)
-  int maxC;     // most CTAs that share one output tile
+  int S;        // row slices of the multiply kernel (grid T x S)
   int S_dense;  // row slices of the dense baseline
   int cl;       // CTAs in the cutoff cluster
   int dense_q16;  // dense-row threshold (share of the row surely used, x 65536)
@@ -78,16 +77,13 @@ effort_status_t make_geometry(int64_t I, int64_t O, Geometry* g) {
     }
   }
   if (g->cl == 0) return EFFORT_ERR_UNSUPPORTED;
-  const long long TU = (long long)g->T * g->G;
-  long long P = (long long)g_num_sms * mac_ctas_per_sm();
-  if (P > TU) P = TU;
-  g->P = (int)P;
-  int maxC = 1;
-  for (long long t = 0; t < g->T; ++t) {  // owner(u) = ((u + 1) * P - 1) / TU
-    const long long cf = ((t * g->G + 1) * P - 1) / TU, cl = (((t + 1) * g->G) * P - 1) / TU;
-    if (cl - cf + 1 > maxC) maxC = (int)(cl - cf + 1);
-  }
-  g->maxC = maxC;
+  // T x S CTAs fill the SMs once (two resident per SM); every slice keeps at
+  // least one 32-row group
+  const int slots = g_num_sms * mac_ctas_per_sm();
+  int S = slots / g->T;
+  if (S < 1) S = 1;
+  if (S > g->G) S = g->G;
+  g->S = S;
   // rows whose surely-used share reaches this fraction are read from the dense
   // copy (2 B per weight, register accumulation) instead of their buckets
   double frac = 0.5;
@@ -106,7 +102,7 @@ effort_status_t make_geometry(int64_t I, int64_t O, Geometry* g) {
 
 // One contiguous device block of scratch for `npairs` jobs.
 effort_status_t alloc_ws(const Geometry& g, int npairs, WsBlock* out, WsPtrs* slots) {
-  const int S = g.maxC > g.S_dense ? g.maxC : g.S_dense;
+  const int S = g.S > g.S_dense ? g.S : g.S_dense;
   const size_t per = align_up(256, 256)                                  // c, count, done, status
                      + align_up((size_t)g.T * 4, 256)                    // tilecnt
                      + align_up((size_t)g.G * 4, 256)                    // gcnt
@@ -343,7 +339,7 @@ effort_status_t effort_gemv_ex(effort_handle_t h, const void* v, effort_dtype_t 
   cudaStream_t s = (cudaStream_t)stream;
   h->last_stream = s;
   cudaError_t e = launch_cutoff(jobs, h->g.I, h->g.cl, s);
-  if (e == cudaSuccess) e = launch_mac(jobs, h->g.P, h->g.maxC, s);
+  if (e == cudaSuccess) e = launch_mac(jobs, h->g.T, h->g.S, s);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return EFFORT_ERR_CUDA;
@@ -362,7 +358,7 @@ effort_status_t effort_gemv_split(effort_handle_t h, const void* v, effort_dtype
   h->last_stream = s;
   cudaError_t e = launch_cutoff(jobs, h->g.I, h->g.cl, s);
   if (e == cudaSuccess) e = cudaEventRecord((cudaEvent_t)mid_event, s);
-  if (e == cudaSuccess) e = launch_mac(jobs, h->g.P, h->g.maxC, s);
+  if (e == cudaSuccess) e = launch_mac(jobs, h->g.T, h->g.S, s);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return EFFORT_ERR_CUDA;
@@ -456,7 +452,7 @@ effort_status_t effort_gemv_batched(effort_workspace_t ws, const effort_handle_t
       if (st != EFFORT_OK) return st;
     }
     cudaError_t e = launch_cutoff_batch(jobs, nj, I, ws->g.cl, s);
-    if (e == cudaSuccess) e = launch_mac_batch(jobs, nj, ws->g.P, ws->g.maxC, s);
+    if (e == cudaSuccess) e = launch_mac_batch(jobs, nj, ws->g.T, ws->g.S, s);
     if (e != cudaSuccess) {
       cudaGetLastError();
       return EFFORT_ERR_CUDA;

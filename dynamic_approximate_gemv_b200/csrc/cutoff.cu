@@ -419,17 +419,42 @@ __global__ void __launch_bounds__(kCutThreads, 1) k_cutoff_dispatch(const __grid
     if (base + warp * kGroupRows < RP && g < G) {
       const unsigned lt = (1u << lane) - 1u;
       const uint4 r4 = make_uint4((unsigned)i, __float_as_uint(vi), tau, (unsigned)ki);
-      if (cls == kClassSparse) {
-        const int p = __popc(bs & lt);
-        rec[(size_t)g * kRecPerGroup + p] = r4;
-        // the read bound of this row in every tile: entries of the tile among the
-        // first min((k+1) H, n) ranks (255 saturates: read the whole bucket)
-        const uint8_t* crow = cntt + ((size_t)i * C + min(ki, C - 1)) * T;
-        unsigned char* urow = ut + (size_t)g * T * 32 + p;
-        for (int t = 0; t < T; ++t) urow[(size_t)t * 32] = crow[t];
-      }
+      if (cls == kClassSparse) rec[(size_t)g * kRecPerGroup + __popc(bs & lt)] = r4;
       if (cls == kClassDense) rec[(size_t)g * kRecPerGroup + 32 + __popc(bd & lt)] = r4;
       if (lane == 0) gcnt[g] = (unsigned)__popc(bs) | ((unsigned)__popc(bd) << 8);
+      // read bounds of the group's sparse rows in every tile: entries of the tile
+      // among the first min((k+1) H, n) ranks (255 saturates: read the whole
+      // bucket).  Each lane loads its row's count row in one batch of 4-byte
+      // loads; then, tile by tile, the 32 lanes store one contiguous 32-byte
+      // line ut[g][t][0..31] (lane = sparse slot).
+      const int p = __popc(bs & lt);
+      const bool sp = cls == kClassSparse;
+      const uint8_t* crow = cntt + ((size_t)i * C + min(ki, C - 1)) * T;
+      unsigned char* ug = ut + (size_t)g * T * 32;
+      for (int t0 = 0; t0 < T; t0 += 32) {
+        unsigned w[8];
+        const int nt = min(32, T - t0);
+        if ((T & 3) == 0) {
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            w[u] = (sp && 4 * u < nt) ? *reinterpret_cast<const unsigned*>(crow + t0 + 4 * u) : 0u;
+        } else {
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            unsigned x = 0u;
+#pragma unroll
+            for (int b = 0; b < 4; ++b)
+              if (sp && 4 * u + b < nt) x |= (unsigned)crow[t0 + 4 * u + b] << (8 * b);
+            w[u] = x;
+          }
+        }
+        // lane p's byte for tile t goes to ug[t * 32 + p]; lanes of unused slots
+        // leave their byte untouched
+#pragma unroll
+        for (int tt = 0; tt < 32; ++tt) {
+          if (tt < nt && sp) ug[(size_t)(t0 + tt) * 32 + p] = (unsigned char)((w[tt >> 2] >> (8 * (tt & 3))) & 0xFFu);
+        }
+      }
     }
   }
   // other CTAs may still be reading this CTA's candidate list
