@@ -55,6 +55,7 @@ def lib():
             "effort_gemv": [vp, vp, f32, vp, vp],
             "effort_gemv_ex": [vp, vp, ctypes.c_int, f32, vp, vp, vp, vp, vp],
             "effort_gemv_split": [vp, vp, ctypes.c_int, f32, vp, vp, vp, vp, vp],
+            "effort_gemv_static": [vp, vp, ctypes.c_int, f32, vp, vp, vp, vp, vp],
             "effort_check": [vp],
             "effort_workspace_create": [i64, i64, i32, ctypes.POINTER(vp)],
             "effort_workspace_destroy": [vp],
@@ -143,6 +144,29 @@ class PreparedMatrix:
                     raise ValueError(f"{nm} must be {dt} of shape {shp}")
         _check(lib().effort_gemv_ex(self._h, _ptr(v), _vdtype(v), ctypes.c_float(effort), _ptr(out), _ptr(cutoff),
                                     _ptr(count), _ptr(rowlen), _stream(v.device)), "effort_gemv")
+        return out
+
+    def gemv_static(self, v, effort, out=None, cutoff=None, count=None, status=None):
+        """gemv whose scratch is the library's fixed per-device array (no device
+        allocation by the library; calls on one device must not overlap).
+        status: optional int32 [1] tensor, set nonzero if v held inf/NaN."""
+        _need_cuda(v, "v")
+        if v.shape != (self.in_dim,):
+            raise ValueError("v has the wrong shape")
+        if out is None:
+            out = torch.empty(self.out_dim, device=v.device, dtype=torch.float32)
+        _need_cuda(out, "out")
+        if out.dtype != torch.float32 or out.shape != (self.out_dim,):
+            raise ValueError("out must be float32 [out_dim]")
+        for t, dt, nm in ((cutoff, torch.float32, "cutoff"), (count, torch.int64, "count"),
+                          (status, torch.int32, "status")):
+            if t is not None:
+                _need_cuda(t, nm)
+                if t.dtype != dt or tuple(t.shape) != (1,):
+                    raise ValueError(f"{nm} must be {dt} of shape (1,)")
+        _check(lib().effort_gemv_static(self._h, _ptr(v), _vdtype(v), ctypes.c_float(effort), _ptr(out),
+                                        _ptr(cutoff), _ptr(count), _ptr(status), _stream(v.device)),
+               "effort_gemv_static")
         return out
 
     def gemv_split(self, v, effort, out, mid_event, stream=None):

@@ -11,7 +11,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libeffort.so")
-SOURCES = ["api.cu", "prep.cu", "cutoff.cu", "mac.cu", "dense.cu"]
+SOURCES = ["api.cu", "prep.cu", "cutoff.cu", "mac.cu", "dense.cu", "noalloc.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 FLAGS = [

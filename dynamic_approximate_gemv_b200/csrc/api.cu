@@ -524,3 +524,28 @@ effort_status_t effort_destroy(effort_handle_t h) {
 }
 
 }  // extern "C"
+
+namespace effort {
+
+// For entry points that bring their own per-call scratch: the handle's device
+// and the launch geometry of one call.
+effort_status_t handle_call_geometry(effort_handle_t h, int* dev, int* I, int* T, int* G, int* S, int* cl) {
+  if (!h) return EFFORT_ERR_ARG;
+  *dev = h->dev;
+  *I = h->g.I;
+  *T = h->g.T;
+  *G = h->g.G;
+  *S = h->g.S;
+  *cl = h->g.cl;
+  return EFFORT_OK;
+}
+
+// The same argument checks and job description as effort_gemv_ex, with the
+// caller's scratch in place of the handle's.
+effort_status_t handle_fill_job(effort_handle_t h, const WsPtrs& ws, const void* v, effort_dtype_t v_dtype,
+                                float effort, float* out, float* cutoff_out, uint64_t* count_out, Job* j) {
+  if (!h) return EFFORT_ERR_ARG;
+  return fill_job(h, ws, v, v_dtype, effort, out, cutoff_out, count_out, nullptr, j);
+}
+
+}  // namespace effort

@@ -55,6 +55,7 @@ typedef enum { EFFORT_F32 = 0, EFFORT_F16 = 1 } effort_dtype_t;
 #define EFFORT_MAX_OUT_DIM 32768      /* a row is sorted inside one thread block */
 #define EFFORT_MAX_IN_DIM 40960       /* the cutoff's chart lives in one cluster's shared memory */
 #define EFFORT_MAX_PAIRS_PER_LAUNCH 16
+#define EFFORT_STATIC_SCRATCH_BYTES (2u << 20) /* per-device scratch of effort_gemv_static */
 
 /*
  * effort_prepare -- the offline pass: `precompute(W)` of the pages.
@@ -112,6 +113,37 @@ effort_status_t effort_gemv_ex(effort_handle_t h, const void* v, effort_dtype_t 
 effort_status_t effort_gemv_split(effort_handle_t h, const void* v, effort_dtype_t v_dtype, float effort,
                                   float* out, float* cutoff_out, uint64_t* count_out, void* mid_event,
                                   void* stream);
+
+/*
+ * effort_gemv_static -- effort_gemv_ex (without rowlen_out) whose per-call
+ *   scratch is a fixed array of EFFORT_STATIC_SCRATCH_BYTES (2 MiB) per device,
+ *   compiled into the library, instead of the handle's workspace.  The pages
+ *   have no counterpart: this is a library service, not part of the method.
+ *   It is for callers that must not allocate device memory on the call path,
+ *   e.g. code running under another component's allocator (a caching
+ *   allocator that must account for every byte, a memory pool sized up
+ *   front), or that needs its device footprint fixed before the first call.
+ *   The call allocates nothing: no cudaMalloc, no cudaFree, no allocating
+ *   library routine.  It issues one cudaMemsetAsync that clears the scratch
+ *   words that must start at zero, the same two kernels as effort_gemv_ex,
+ *   and, if status_out is given, one 4-byte device-to-device copy.
+ *   v, v_dtype, effort, out, cutoff_out, count_out: as for effort_gemv_ex.
+ *   status_out: nullable device uint32; receives 0 if the call saw only
+ *     finite entries of v and no internal inconsistency, nonzero otherwise
+ *     (the output is then unspecified).  effort_check does not see this call.
+ *   Set-up: the first call on a device looks up that device's copy of the
+ *     array (cudaGetSymbolAddress, with the handle's device made current);
+ *     make that first call before any stream capture on the device.
+ *   Every call on one device shares the array: calls that may overlap on the
+ *     GPU (unordered streams, concurrent host threads) race and give wrong
+ *     results; order them on one stream.
+ *   Returns EFFORT_ERR_UNSUPPORTED when the handle's geometry needs more than
+ *     EFFORT_STATIC_SCRATCH_BYTES of scratch (4096 x 14336 needs about 0.6 MiB,
+ *     14336 x 4096 about 1 MiB), and when the device ordinal is 64 or above.
+ */
+effort_status_t effort_gemv_static(effort_handle_t h, const void* v, effort_dtype_t v_dtype, float effort,
+                                   float* out, float* cutoff_out, uint64_t* count_out, uint32_t* status_out,
+                                   void* stream);
 
 /*
  * effort_check -- synchronises the handle's last stream and reports whether a
