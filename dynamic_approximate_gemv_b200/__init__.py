@@ -206,7 +206,7 @@ class PreparedMatrix:
             "vals": view(L.vals, (T, I, cap), "<i2"), "idx": view(L.idx, (T, I, cap), "|u1"),
             "probes": view(L.probes, (I, L.n_probes), "<i2"), "ckmag": view(L.ckmag, (I, C + 1), "<i2"),
             "cnt": view(L.cnt, (I, C, T), "|u1"), "wdense": view(L.wdense, (I, T * 256), "<i2"),
-            "rec": view(L.rec, (L.n_groups, 64, 4), "<u4"), "gcnt": view(L.gcnt, (L.n_groups,), "<u4"),
+            "rec": view(L.rec, (L.n_groups, 32, 2), "<u4"), "gcnt": view(L.gcnt, (L.n_groups,), "<u4"),
         }
 
     def close(self):

@@ -107,7 +107,7 @@ effort_status_t alloc_ws(const Geometry& g, int npairs, WsBlock* out, WsPtrs* sl
                      + align_up((size_t)g.T * 4, 256)                    // tilecnt
                      + align_up((size_t)g.G * 4, 256)                    // gcnt
                      + align_up((size_t)g.G * g.T * 32, 256)             // ut
-                     + align_up((size_t)g.G * kRecPerGroup * 16, 256)    // rec
+                     + align_up((size_t)g.G * kRecPerGroup * 8, 256)     // rec
                      + align_up((size_t)S * g.T * kTW * 4, 256);         // part
   const size_t bytes = per * (size_t)npairs;
   void* base = nullptr;
@@ -133,8 +133,8 @@ effort_status_t alloc_ws(const Geometry& g, int npairs, WsBlock* out, WsPtrs* sl
     b += align_up((size_t)g.G * 4, 256);
     w.ut = (unsigned char*)b;
     b += align_up((size_t)g.G * g.T * 32, 256);
-    w.rec = (uint4*)b;
-    b += align_up((size_t)g.G * kRecPerGroup * 16, 256);
+    w.rec = (uint2*)b;
+    b += align_up((size_t)g.G * kRecPerGroup * 8, 256);
     w.part = (float*)b;
     slots[p] = w;
   }

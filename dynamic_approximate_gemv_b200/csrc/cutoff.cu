@@ -25,7 +25,8 @@
 //           dense fraction, 1/2 by default) are "dense" (read from the dense
 //           copy), other active rows are "sparse" (read from the sorted
 //           buckets), rows whose largest product is below c are off.  Records
-//           {row, v_i, tau_i, k_i} go to fixed slots of their 32-row group.
+//           {v_i, tau_i, row} of a 32-row group are written sparse rows first,
+//           then dense rows.
 #include <cooperative_groups.h>
 
 #include "effort_internal.cuh"
@@ -161,7 +162,7 @@ __global__ void __launch_bounds__(kCutThreads, 1) k_cutoff_dispatch(const __grid
   const void* vptr = jb.v;
   const int vdtype = jb.vdtype, dense_q16 = jb.dense_q16;
   unsigned* __restrict__ status = jb.ws.status;
-  uint4* __restrict__ rec = jb.ws.rec;
+  uint2* __restrict__ rec = jb.ws.rec;
   unsigned* __restrict__ gcnt = jb.ws.gcnt;
   unsigned char* __restrict__ ut = jb.ws.ut;
   const uint8_t* __restrict__ cntt = jb.hd.cnt;
@@ -418,9 +419,9 @@ __global__ void __launch_bounds__(kCutThreads, 1) k_cutoff_dispatch(const __grid
     // a group is written only by the CTA whose row range holds it
     if (base + warp * kGroupRows < RP && g < G) {
       const unsigned lt = (1u << lane) - 1u;
-      const uint4 r4 = make_uint4((unsigned)i, __float_as_uint(vi), tau, (unsigned)ki);
-      if (cls == kClassSparse) rec[(size_t)g * kRecPerGroup + __popc(bs & lt)] = r4;
-      if (cls == kClassDense) rec[(size_t)g * kRecPerGroup + 32 + __popc(bd & lt)] = r4;
+      const uint2 r2 = make_uint2(__float_as_uint(vi), (tau & 0xFFFFu) | ((unsigned)i << 16));
+      if (cls == kClassSparse) rec[(size_t)g * kRecPerGroup + __popc(bs & lt)] = r2;
+      if (cls == kClassDense) rec[(size_t)g * kRecPerGroup + __popc(bs) + __popc(bd & lt)] = r2;
       if (lane == 0) gcnt[g] = (unsigned)__popc(bs) | ((unsigned)__popc(bd) << 8);
       // read bounds of the group's sparse rows in every tile: entries of the tile
       // among the first min((k+1) H, n) ranks (255 saturates: read the whole

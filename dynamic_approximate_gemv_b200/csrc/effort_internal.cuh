@@ -32,7 +32,7 @@ constexpr int kPrepThreads = 1024;
 constexpr int kDenseThreads = 256;
 constexpr int kMaxJobs = 16;     // pairs per launch
 constexpr int kGroupRows = 32;   // dispatch records are grouped by 32 rows
-constexpr int kRecPerGroup = 64; // 32 sparse slots + 32 dense slots
+constexpr int kRecPerGroup = 32; // one 8-byte record per row of a group
 
 // call modes decided on the host from K and the kept count
 enum : int { kModeSelect = 0, kModeAll = 1, kModeNone = 2 };
@@ -62,8 +62,9 @@ struct WsPtrs {
   unsigned long long* count;    // running |S|
   unsigned int* done;           // CTAs of the multiply kernel that finished
   unsigned int* tilecnt;        // [T] split-K arrivals per tile
-  uint4* rec;                   // [G][64] dispatch records {row, v bits, tau (fp16 bits), k}
-  unsigned int* gcnt;           // [G] (#sparse) | (#dense << 8)
+  uint2* rec;                   // [G][32] dispatch records {v bits, tau (fp16 bits) | row << 16}:
+                                //   sparse rows at [0, ns), dense rows at [ns, ns + nd)
+  unsigned int* gcnt;           // [G] ns | nd << 8
   unsigned char* ut;            // [G][T][32]: read bound U of sparse slot p of group g in tile t
   float* part;                  // per-tile partial sums of the CTAs that share a tile
   unsigned int* status;         // sticky device status bits

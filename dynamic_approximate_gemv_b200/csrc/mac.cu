@@ -8,73 +8,86 @@
 // Selection test.  For row i the dispatch computed tau_i, the smallest fp16
 // magnitude m with fl32(|v_i| * m) >= c.  Because fl32(a * m) does not
 // decrease as m grows, "|w| >= tau_i" holds exactly for the weights whose
-// product passes the cutoff; the kernel compares magnitudes and never forms
-// the compare product.
+// product passes the cutoff; the kernel compares fp16 magnitudes (two per
+// instruction) and never forms the compare product.
 //
 // Work split.  CTA (t, s) of a T x S grid owns output tile t and the 32-row
-// groups [s*G/S, (s+1)*G/S).  It stages the dispatch records of its groups in
-// shared memory (16 groups per round, one round of loads each), then streams
-// the rows:
+// groups [s*G/S, (s+1)*G/S).  It stages the dispatch records of up to 32
+// groups per round in shared memory (one warp per group, two block barriers
+// per round), then streams the rows:
 //   dense rows   the row's 256 weights of the tile come from the dense copy
-//                and are accumulated in registers, 8 columns per lane, with a
-//                predicated FMA;
+//                and are accumulated in registers, 8 columns per lane: a
+//                packed magnitude mask zeroes the unused weights, then a
+//                packed fp32 FMA adds v_i * w;
 //   sparse rows  the bucket's leading U entries (U from the dispatch's read
-//                bound table) are cut into chunks of up to 64 entries; a ring
-//                slot holds two chunks and each half-warp scatters one of them,
-//                4 entries per lane, into its own shared copy of the tile.  The
-//                entries of one bucket have distinct columns, so a half-warp
-//                updates its copy with plain loads and stores; a __syncwarp
-//                separates slots.
-// Each warp streams its items through a ring of 512 B slots in shared memory
-// filled with cp.async (16 B per lane), so several items per warp are in
-// flight without holding registers.  At the end a CTA sums its warp copies and
-// registers into one partial tile; the last of the S CTAs of a tile to arrive
-// adds the partials in slice order (no float atomics: results are
-// reproducible run to run).
+//                bound table) are cut into chunks of up to 32 entries.  A work
+//                item holds four chunks; each half-warp takes two of them in
+//                turn, 2 entries per lane, and adds the selected products into
+//                its own shared copy of the tile.  The entries of one bucket
+//                have distinct columns, so a half-warp updates its copy with
+//                plain loads and stores; a __syncwarp separates its chunks.
+// Each warp streams its items through a ring of 512-byte slots in shared
+// memory filled with cp.async (16 bytes per lane; bytes past a chunk's end are
+// zero-filled by the copy), so several items per warp are in flight without
+// holding registers.  At the end a CTA sums its warp copies and registers into
+// one partial tile; the last of the S CTAs of a tile to arrive adds the
+// partials in slice order (no float atomics: results are reproducible run to
+// run).
 #include "effort_internal.cuh"
 
 namespace effort {
 
 constexpr int kSlots = 6;
-constexpr int kSlotBytes = 512;    // one dense tile-row, or two chunks (64 values + 64 columns each)
-constexpr int kChunk = 64;         // bucket entries per sparse chunk
-constexpr int kSegGroups = 16;     // groups staged per round
-constexpr int kSegRecs = kSegGroups * 32;
-constexpr int kMaxChunks = 1024;   // a round takes only the leading groups whose chunks fit
-constexpr int kStagePairs = (kSegGroups * kRecPerGroup + kMacThreads - 1) / kMacThreads;
+constexpr int kSlotBytes = 512;     // one dense tile row, or four chunks
+constexpr int kChunk = 32;          // bucket entries per sparse chunk
+constexpr int kChunkBytes = 128;    // 64 B values, 32 B columns, 32 B unused
+constexpr int kRoundGroups = 32;    // groups staged per round (two per warp)
+constexpr int kRoundRows = kRoundGroups * 32;
+constexpr int kMaxChunks = 1280;    // a round takes only the leading groups whose chunks fit
 
-// Staged work.  dense rows: {first element of the row's tile in the dense
-// copy, v bits, tau as float bits, row}; sparse chunks: {first entry of the
-// chunk, v bits, tau as float bits, entries in the chunk | row << 8}.
+// Staged work of one round:
+//   dense row  {v bits, tau | row << 16}
+//   chunk      {first entry, entries, v bits, tau | row << 16}; the list is
+//              padded to whole items with empty chunks (no entries, tau = +inf)
 struct MacSmem {
   float acc[kMacWarps][2][kTW];  // a shared copy of the tile per half-warp
-  uint4 recD[kSegRecs];
+  uint2 recD[kRoundRows];
   uint4 chunk[kMaxChunks];
-  unsigned short nchk[kSegRecs];  // chunks of each staged sparse row, then their start
-  int offD[kSegGroups + 1];
-  int offS[kSegGroups + 1];
-  unsigned warp_tot[kMacWarps];
+  int gtot[2][kRoundGroups];     // per staged group: dense rows, chunks
   unsigned long long warp_cnt[kMacWarps];
-  int nchunks;
-  int ngroups;  // groups the round takes
   int flag;
   alignas(16) unsigned char ring[kMacWarps][kSlots][kSlotBytes];
 };
 
-__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
-  const unsigned dst = (unsigned)__cvta_generic_to_shared(smem_dst);
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(gsrc) : "memory");
+__device__ __forceinline__ unsigned smem_u32(const void* p) { return (unsigned)__cvta_generic_to_shared(p); }
+// Streamed weights are read once per call: they are copied with an L2
+// evict-first policy so that they do not push the kernels' code, the dispatch
+// records and the tables out of L2.
+__device__ __forceinline__ unsigned long long evict_first_policy() {
+  unsigned long long p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ void cp_async16(unsigned dst, const void* gsrc, unsigned long long pol) {
+  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, 16, %2;\n" ::"r"(dst), "l"(gsrc), "l"(pol)
+               : "memory");
 }
 // copies `bytes` (0..16) and zero-fills the rest of the 16-byte destination
-__device__ __forceinline__ void cp_async16_zfill(void* smem_dst, const void* gsrc, unsigned bytes) {
-  const unsigned dst = (unsigned)__cvta_generic_to_shared(smem_dst);
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(gsrc), "r"(bytes) : "memory");
+__device__ __forceinline__ void cp_async16_zfill(unsigned dst, const void* gsrc, unsigned bytes, unsigned long long pol) {
+  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;\n" ::"r"(dst), "l"(gsrc), "r"(bytes),
+               "l"(pol) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
+// mask with 0xFFFF in each half whose magnitude is >= tau (both halves hold tau)
+__device__ __forceinline__ unsigned ge_mask(unsigned w2, unsigned tau2) {
+  const unsigned mag = w2 & 0x7FFF7FFFu;
+  return __hge2_mask(*reinterpret_cast<const __half2*>(&mag), *reinterpret_cast<const __half2*>(&tau2));
+}
+
 
 template <int NJ, bool STATS>
 __global__ void __launch_bounds__(kMacThreads, 2) k_mac(const __grid_constant__ Jobs<NJ> jobs, int S) {
@@ -89,7 +102,7 @@ __global__ void __launch_bounds__(kMacThreads, 2) k_mac(const __grid_constant__ 
   const int dstride = jb.hd.dstride;
   const unsigned long long kept_total = jb.hd.kept_total;
   const unsigned* __restrict__ gcnt = jb.ws.gcnt;
-  const uint4* __restrict__ grec_all = jb.ws.rec;
+  const uint2* __restrict__ grec_all = jb.ws.rec;
   const unsigned char* __restrict__ ut = jb.ws.ut;
   float* __restrict__ part_all = jb.ws.part;
   unsigned* tilecnt = jb.ws.tilecnt;
@@ -108,243 +121,243 @@ __global__ void __launch_bounds__(kMacThreads, 2) k_mac(const __grid_constant__ 
   const float c = *reinterpret_cast<volatile float*>(jb.ws.c);
   const bool count_all = (__float_as_uint(c) == 0u);
   const bool want_rowlen = STATS && rowlen_out != nullptr && !count_all;
-  float a8[8];
+  float2 acc2[4];
 #pragma unroll
-  for (int m = 0; m < 8; ++m) a8[m] = 0.0f;
+  for (int u = 0; u < 4; ++u) acc2[u] = make_float2(0.0f, 0.0f);
   unsigned nsel = 0;
   unsigned char* ring = sh.ring[warp][0];
+  const unsigned ring_base = smem_u32(ring);
+  const unsigned long long pol = evict_first_policy();
+  const int h = lane >> 4, hl = lane & 15;
+  float* acc_h = sh.acc[warp][h];
+  // copy roles for a sparse item: chunk cp_ck = lane / 6 (lanes 0..23); four
+  // lanes copy its 64 value bytes, two lanes its 32 column bytes
+  const int cp_ck = lane / 6, cp_r = lane - 6 * (lane / 6);
+  const bool cp_val = cp_r < 4;
+  const int cp_sub = cp_val ? cp_r : cp_r - 4;
+  const bool cp_act = lane < 24;
+  const unsigned cp_dst = (unsigned)(kChunkBytes * cp_ck + (cp_val ? 16 * cp_sub : 64 + 16 * cp_sub));
+  // source of lane's 16 bytes: base + first * mul, valid bytes len * mul - 16 sub
+  const char* cp_base = cp_val ? reinterpret_cast<const char*>(vals) + 16 * cp_sub
+                               : reinterpret_cast<const char*>(idxs) + 16 * cp_sub;
+  const unsigned cp_mul = cp_val ? 2u : 1u;
+  const int cp_off = 16 * cp_sub;
 
-  {
-    for (int q0 = gb; q0 < ge; q0 += sh.ngroups) {
-      const int ng_load = min(kSegGroups, ge - q0);
-      // ---- stage: one round of independent loads (counts, records, read bounds)
-      uint4 r4[kStagePairs];
-      unsigned u8v[kStagePairs];
+  for (int q0 = gb; q0 < ge;) {
+    const int ng_load = min(kRoundGroups, ge - q0);
+    // ---- stage: warp w reads groups q0 + w and q0 + w + 16 (records, read
+    // bounds and counts in one round of loads; records past a group's counts
+    // are stale and ignored)
+    uint2 rr[2];
+    unsigned uu[2], gc[2];
 #pragma unroll
-      for (int z = 0; z < kStagePairs; ++z) {
-        const int pr = threadIdx.x + z * kMacThreads;  // (group, slot) pair
-        const int gq = pr >> 6, p = pr & 63;
-        r4[z] = make_uint4(0, 0, 0, 0);
-        u8v[z] = 0;
-        if (gq < ng_load) {
-          r4[z] = grec_all[(size_t)(q0 + gq) * kRecPerGroup + p];
-          if (p < 32) u8v[z] = ut[((size_t)(q0 + gq) * T + t) * 32 + p];
-        }
+    for (int z = 0; z < 2; ++z) {
+      const int gq = warp + kMacWarps * z;
+      rr[z] = make_uint2(0, 0);
+      uu[z] = gc[z] = 0;
+      if (gq < ng_load) {
+        const size_t g = (size_t)(q0 + gq);
+        gc[z] = gcnt[g];
+        rr[z] = grec_all[g * kRecPerGroup + lane];
+        uu[z] = ut[(g * T + t) * 32 + lane];
       }
-      if (warp == 0) {
-        unsigned gc = 0;
-        if (lane < ng_load) gc = gcnt[q0 + lane];
-        int is = (int)(gc & 0xFFu), id = (int)((gc >> 8) & 0xFFu);
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int ys = __shfl_up_sync(0xFFFFFFFFu, is, o), yd = __shfl_up_sync(0xFFFFFFFFu, id, o);
-          if (lane >= o) {
-            is += ys;
-            id += yd;
-          }
-        }
-        if (lane < kSegGroups) {
-          sh.offS[lane + 1] = is;
-          sh.offD[lane + 1] = id;
-        }
-        if (lane == 0) sh.offS[0] = sh.offD[0] = 0;
-      }
-      __syncthreads();
-      // dense rows go to their list; sparse rows note how many chunks they need
-#pragma unroll
-      for (int z = 0; z < kStagePairs; ++z) {
-        const int pr = threadIdx.x + z * kMacThreads;
-        const int gq = pr >> 6, p = pr & 63;
-        if (gq < ng_load) {
-          if (p < 32) {
-            if (p < sh.offS[gq + 1] - sh.offS[gq]) {
-              const unsigned U = (u8v[z] == 255u) ? (unsigned)kCap : u8v[z];
-              sh.nchk[sh.offS[gq] + p] = (unsigned short)((U + kChunk - 1) / kChunk);
-            }
-          } else if (p - 32 < sh.offD[gq + 1] - sh.offD[gq]) {
-            const uint4 r = r4[z];
-            const float tau = __half2float(__ushort_as_half((unsigned short)r.z));
-            sh.recD[sh.offD[gq] + p - 32] =
-                make_uint4((unsigned)((size_t)r.x * dstride + (size_t)t * kTW), r.y, __float_as_uint(tau), r.x);
-          }
-        }
-      }
-      __syncthreads();
-      const int NS = sh.offS[ng_load];
-      {  // exclusive scan of the chunk counts (NS <= kSegRecs <= kMacThreads)
-        unsigned x = (threadIdx.x < NS) ? sh.nchk[threadIdx.x] : 0u;
-        unsigned incl = x;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const unsigned y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-          if (lane >= o) incl += y;
-        }
-        if (lane == 31) sh.warp_tot[warp] = incl;
-        __syncthreads();
-        unsigned before = 0;
-        for (int w = 0; w < warp; ++w) before += sh.warp_tot[w];
-        if (threadIdx.x < NS) sh.nchk[threadIdx.x] = (unsigned short)(before + incl - x);
-        if (threadIdx.x == kMacThreads - 1) sh.nchunks = (int)(before + incl);
-      }
-      __syncthreads();
-      if (threadIdx.x == 0) {  // the leading groups whose chunks fit the chunk list
-        int take = ng_load, nc = sh.nchunks;
-        while (nc > kMaxChunks) {
-          --take;
-          nc = (sh.offS[take] < NS) ? (int)sh.nchk[sh.offS[take]] : sh.nchunks;
-        }
-        sh.ngroups = take;
-        sh.nchunks = nc;
-      }
-      __syncthreads();
-      const int ng = sh.ngroups;
-      // sparse rows: their chunks go to the chunk list
-#pragma unroll
-      for (int z = 0; z < kStagePairs; ++z) {
-        const int pr = threadIdx.x + z * kMacThreads;
-        const int gq = pr >> 6, p = pr & 63;
-        if (gq < ng && p < 32 && p < sh.offS[gq + 1] - sh.offS[gq]) {
-          const uint4 r = r4[z];
-          const unsigned U = (u8v[z] == 255u) ? (unsigned)kCap : u8v[z];
-          const float tau = __half2float(__ushort_as_half((unsigned short)r.z));
-          const unsigned first = (unsigned)(((size_t)t * I + r.x) * kCap);
-          int slot = sh.nchk[sh.offS[gq] + p];
-          for (unsigned e0 = 0; e0 < U; e0 += kChunk, ++slot)
-            sh.chunk[slot] = make_uint4(first + e0, r.y, __float_as_uint(tau), min(U - e0, (unsigned)kChunk) | (r.x << 8));
-        }
-      }
-      __syncthreads();
-      const int ND = sh.offD[ng];
-      const int NC = sh.nchunks;
-      const int NI = ND + (NC + 1) / 2;  // dense rows, then pairs of chunks
-      // this warp's items: j = warp, warp + NW, ...
-      const int nmine = (NI > warp) ? (NI - warp + kMacWarps - 1) / kMacWarps : 0;
-
-      // A pair slot holds two chunks: values at [256 h, 256 h + 128), columns at
-      // [256 h + 128, 256 h + 192).  Lanes 0..15 copy values (8 per chunk), lanes
-      // 16..23 copy columns (4 per chunk); bytes past a chunk's length are
-      // zero-filled, so those entries carry weight 0 and never pass tau > 0.
-      const bool cp_val = lane < 16;
-      const int cp_h = cp_val ? (lane >> 3) : ((lane - 16) >> 2);
-      const int cp_k = cp_val ? (lane & 7) : ((lane - 16) & 3);
-      const int cp_dst = 256 * cp_h + (cp_val ? 16 * cp_k : 128 + 16 * cp_k);
-      auto issue = [&](int q) {  // the warp's q-th item into ring slot q % kSlots
-        if (q < nmine) {
-          const int j = warp + q * kMacWarps;
-          unsigned char* slot = ring + (q % kSlots) * kSlotBytes;
-          if (j < ND) {
-            cp_async16(slot + 16 * lane, wdense + sh.recD[j].x + 8 * lane);
-          } else if (lane < 24) {
-            const int ch = 2 * (j - ND) + cp_h;
-            const uint4 r = (ch < NC) ? sh.chunk[ch] : make_uint4(0, 0, 0, 0);
-            const int len = (int)(r.w & 0xFFu);
-            const int nb = cp_val ? 2 * len - 16 * cp_k : len - 16 * cp_k;
-            const void* src = cp_val ? (const void*)(vals + r.x + 8 * cp_k) : (const void*)(idxs + r.x + 16 * cp_k);
-            cp_async16_zfill(slot + cp_dst, src, (unsigned)max(0, min(16, nb)));
-          }
-        }
-        cp_async_commit();
-      };
-
-#pragma unroll
-      for (int q = 0; q < kSlots - 1; ++q) issue(q);
-      for (int q = 0; q < nmine; ++q) {
-        cp_async_wait<kSlots - 2>();
-        __syncwarp();
-        const int j = warp + q * kMacWarps;
-        const unsigned char* slot = ring + (q % kSlots) * kSlotBytes;
-        if (j < ND) {
-          const uint4 r = sh.recD[j];
-          const float vi = __uint_as_float(r.y), tau = __uint_as_float(r.z);
-          const uint4 wv = *reinterpret_cast<const uint4*>(slot + 16 * lane);
-          const __half* h = reinterpret_cast<const __half*>(&wv);
-          unsigned rs = 0;
-#pragma unroll
-          for (int m = 0; m < 8; ++m) {
-            const float w = __half2float(h[m]);
-            const bool sel = fabsf(w) >= tau;
-            a8[m] = sel ? fmaf(vi, w, a8[m]) : a8[m];
-            if (STATS) rs += sel ? 1u : 0u;
-          }
-          if (STATS) {
-            nsel += rs;
-            if (want_rowlen) {
-#pragma unroll
-              for (int o = 16; o > 0; o >>= 1) rs += __shfl_xor_sync(0xFFFFFFFFu, rs, o);
-              if (lane == 0 && rs) atomicAdd(&rowlen_out[r.w], rs);
-            }
-          }
-        } else {
-          // half-warp h scatters chunk 2 (j - ND) + h, 4 entries per lane
-          const int h = lane >> 4, hl = lane & 15;
-          const int ch = 2 * (j - ND) + h;
-          const uint4 r = (ch < NC) ? sh.chunk[ch] : make_uint4(0, 0, 0x7F800000u, 0);  // missing: tau = inf
-          const float vi = __uint_as_float(r.y), tau = __uint_as_float(r.z);
-          const uint2 w4 = *reinterpret_cast<const uint2*>(slot + 256 * h + 8 * hl);
-          const unsigned c4 = *reinterpret_cast<const unsigned*>(slot + 256 * h + 128 + 4 * hl);
-          const __half* hw = reinterpret_cast<const __half*>(&w4);
-          float* acc = sh.acc[warp][h];
-          unsigned rs = 0;
-#pragma unroll
-          for (int m = 0; m < 4; ++m) {
-            const float w = __half2float(hw[m]);
-            const bool sel = fabsf(w) >= tau;
-            float* a = acc + ((c4 >> (8 * m)) & 255u);
-            const float nv = fmaf(vi, w, *a);
-            if (sel) *a = nv;
-            if (STATS) rs += sel ? 1u : 0u;
-          }
-          if (STATS) {
-            nsel += rs;
-            if (want_rowlen) {
-#pragma unroll
-              for (int o = 8; o > 0; o >>= 1) rs += __shfl_xor_sync(0xFFFFFFFFu, rs, o);
-              if (hl == 0 && rs) atomicAdd(&rowlen_out[r.w >> 8], rs);
-            }
-          }
-        }
-        __syncwarp();  // slot and tile copies are free for the next item
-        issue(q + kSlots - 1);
-      }
-      cp_async_wait<0>();
-      __syncthreads();  // the next round's staging overwrites this round's lists
     }
-
-    // ---- leave tile t: one partial tile per CTA, summed in CTA order by the last to arrive
+    int nck[2], cincl[2];
 #pragma unroll
-    for (int m = 0; m < 8; ++m) {
-      sh.acc[warp][0][8 * lane + m] += a8[m];
-      a8[m] = 0.0f;
+    for (int z = 0; z < 2; ++z) {
+      const int gq = warp + kMacWarps * z;
+      const int ns = (int)(gc[z] & 0xFFu), nd = (int)((gc[z] >> 8) & 0xFFu);
+      const unsigned U = (uu[z] == 255u) ? (unsigned)kCap : uu[z];
+      nck[z] = (lane < ns) ? (int)((U + kChunk - 1) / kChunk) : 0;
+      int x = nck[z];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+        if (lane >= o) x += y;
+      }
+      cincl[z] = x;
+      if (lane == 31 && gq < ng_load) {
+        sh.gtot[0][gq] = nd;
+        sh.gtot[1][gq] = x;
+      }
     }
     __syncthreads();
-    float s = 0.0f;
-    if (threadIdx.x < kTW) {
+    // every warp: offsets of the staged groups, and how many leading groups
+    // the round takes (their chunks must fit the chunk list)
+    int od = (lane < ng_load) ? sh.gtot[0][lane] : 0;
+    int oc = (lane < ng_load) ? sh.gtot[1][lane] : 0;
 #pragma unroll
-      for (int w = 0; w < kMacWarps; ++w) {
-        s += sh.acc[w][0][threadIdx.x] + sh.acc[w][1][threadIdx.x];
-        sh.acc[w][0][threadIdx.x] = 0.0f;
-        sh.acc[w][1][threadIdx.x] = 0.0f;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int yd = __shfl_up_sync(0xFFFFFFFFu, od, o);
+      const int yc = __shfl_up_sync(0xFFFFFFFFu, oc, o);
+      if (lane >= o) {
+        od += yd;
+        oc += yc;
       }
     }
-    const int col = t * kTW + threadIdx.x;
-    if (S == 1) {
-      if (threadIdx.x < kTW && col < O) out[col] = s;
-    } else {
-      float* part = part_all + (size_t)t * S * kTW;
-      if (threadIdx.x < kTW) part[(size_t)sl * kTW + threadIdx.x] = s;
-      __threadfence();
-      __syncthreads();
-      if (threadIdx.x == 0) sh.flag = (atomicAdd(&tilecnt[t], 1u) == (unsigned)(S - 1));
-      __syncthreads();
-      if (sh.flag) {
-        __threadfence();
-        if (threadIdx.x < kTW) {
-          float tot = 0.0f;
-          for (int k = 0; k < S; ++k) tot += __ldcg(&part[(size_t)k * kTW + threadIdx.x]);
-          if (col < O) out[col] = tot;
+    const unsigned over = __ballot_sync(0xFFFFFFFFu, lane < ng_load && oc > kMaxChunks - 3);
+    const int take = over ? (__ffs(over) - 1) : ng_load;  // >= 1: one group has at most 256 chunks
+    const int ND = __shfl_sync(0xFFFFFFFFu, od, take - 1);
+    const int NC0 = __shfl_sync(0xFFFFFFFFu, oc, take - 1);  // chunks of the taken groups
+    const int NC = (NC0 + 3) & ~3;                            // padded to whole items
+#pragma unroll
+    for (int z = 0; z < 2; ++z) {
+      const int gq = warp + kMacWarps * z;
+      if (gq < take) {  // warp-uniform
+        const int src = gq > 0 ? gq - 1 : 0;
+        const int xd = __shfl_sync(0xFFFFFFFFu, od, src), xc = __shfl_sync(0xFFFFFFFFu, oc, src);
+        const int offD = gq > 0 ? xd : 0, offC = gq > 0 ? xc : 0;
+        const int ns = (int)(gc[z] & 0xFFu), nd = (int)((gc[z] >> 8) & 0xFFu);
+        if (lane >= ns && lane < ns + nd) sh.recD[offD + lane - ns] = rr[z];
+        if (lane < ns) {
+          const unsigned U = (uu[z] == 255u) ? (unsigned)kCap : uu[z];
+          const unsigned first = (unsigned)(((size_t)t * I + (rr[z].y >> 16)) * kCap);
+          const int cpos = offC + cincl[z] - nck[z];
+          for (int k = 0; k < nck[z]; ++k)
+            sh.chunk[cpos + k] = make_uint4(first + (unsigned)(k * kChunk), min(U - (unsigned)(k * kChunk), (unsigned)kChunk),
+                                            rr[z].x, rr[z].y);
         }
-        if (threadIdx.x == 0) tilecnt[t] = 0u;
       }
+    }
+    if (threadIdx.x < NC - NC0) sh.chunk[NC0 + threadIdx.x] = make_uint4(0u, 0u, 0u, 0x7C00u);
+    __syncthreads();
+    const int NI = ND + NC / 4;  // dense rows, then items of four chunks
+    // this warp's items: j = warp + 16 q; dense while q < nmineD
+    const int nmine = (NI > warp) ? (NI - warp + kMacWarps - 1) / kMacWarps : 0;
+    const int nmineD = (ND > warp) ? (ND - warp + kMacWarps - 1) / kMacWarps : 0;
+
+    // sparse item j: lanes 0..23 copy their 16 bytes of chunk 4 (j - ND) + cp_ck
+    auto issue_sparse = [&](int j, unsigned dst) {
+      if (cp_act) {
+        const uint2 r = *reinterpret_cast<const uint2*>(&sh.chunk[4 * (j - ND) + cp_ck]);  // {first, entries}
+        const int nb = min(16, max(0, (int)(r.y * cp_mul) - cp_off));
+        cp_async16_zfill(dst + cp_dst, cp_base + (size_t)r.x * cp_mul, (unsigned)nb, pol);
+      }
+    };
+    auto issue = [&](int q, unsigned dst) {  // the warp's q-th item into the ring slot at dst
+      const int j = warp + q * kMacWarps;
+      if (q < nmineD) {
+        const unsigned row = sh.recD[j].y >> 16;
+        cp_async16(dst + 16 * lane, wdense + (size_t)row * dstride + (size_t)t * kTW + 8 * lane, pol);
+      } else if (q < nmine) {
+        issue_sparse(j, dst);
+      }
+      cp_async_commit();
+    };
+    constexpr unsigned kRingLast = (kSlots - 1) * kSlotBytes;
+    unsigned so_i = 0, so_p = 0;  // byte offsets of the next slot to fill and to process
+#pragma unroll
+    for (int q = 0; q < kSlots - 1; ++q) {
+      issue(q, ring_base + so_i);
+      so_i = (so_i == kRingLast) ? 0u : so_i + kSlotBytes;
+    }
+    int q = 0;
+    // dense items: 8 columns per lane, accumulated in registers
+    for (; q < nmineD; ++q) {
+      cp_async_wait<kSlots - 2>();
+      __syncwarp();
+      const uint2 r = sh.recD[warp + q * kMacWarps];
+      const float vi = __uint_as_float(r.x);
+      const unsigned tau2 = (r.y & 0xFFFFu) * 0x10001u;
+      const uint4 wv = *reinterpret_cast<const uint4*>(ring + so_p + 16 * lane);
+      const unsigned wr[4] = {wv.x, wv.y, wv.z, wv.w};
+      const float2 v2 = make_float2(vi, vi);
+      unsigned rsel = 0;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const unsigned m = ge_mask(wr[u], tau2);
+        const unsigned wk = wr[u] & m;  // unused weights become +0
+        acc2[u] = __ffma2_rn(v2, __half22float2(*reinterpret_cast<const __half2*>(&wk)), acc2[u]);
+        if (STATS) rsel += (unsigned)__popc(m) >> 4;
+      }
+      if (STATS) {
+        nsel += rsel;
+        if (want_rowlen) {
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) rsel += __shfl_xor_sync(0xFFFFFFFFu, rsel, o);
+          if (lane == 0 && rsel) atomicAdd(&rowlen_out[r.y >> 16], rsel);
+        }
+      }
+      __syncwarp();  // the slot is free for the next copy
+      issue(q + kSlots - 1, ring_base + so_i);
+      so_i = (so_i == kRingLast) ? 0u : so_i + kSlotBytes;
+      so_p = (so_p == kRingLast) ? 0u : so_p + kSlotBytes;
+    }
+    // sparse items: half-warp h takes chunks 2h and 2h + 1 of the item in turn,
+    // 2 entries per lane
+    for (; q < nmine; ++q) {
+      cp_async_wait<kSlots - 2>();
+      __syncwarp();
+      const int cb0 = 4 * (warp + q * kMacWarps - ND) + 2 * h;
+#pragma unroll
+      for (int kk = 0; kk < 2; ++kk) {
+        const uint2 rr = *reinterpret_cast<const uint2*>(&sh.chunk[cb0 + kk].z);  // {v bits, tau | row << 16}
+        const unsigned char* cb = ring + so_p + kChunkBytes * (2 * h + kk);
+        const float vi = __uint_as_float(rr.x);
+        const unsigned tau2 = (rr.y & 0xFFFFu) * 0x10001u;
+        const unsigned w2 = *reinterpret_cast<const unsigned*>(cb + 4 * hl);
+        const unsigned ix = *reinterpret_cast<const unsigned short*>(cb + 64 + 2 * hl);
+        const unsigned m = ge_mask(w2, tau2);  // zero-filled entries have w = 0 < tau
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w2));
+        if (m & 0xFFFFu) {
+          float* a = acc_h + (ix & 0xFFu);
+          *a = fmaf(vi, f.x, *a);
+        }
+        if (m >> 16) {
+          float* a = acc_h + (ix >> 8);
+          *a = fmaf(vi, f.y, *a);
+        }
+        if (STATS) {
+          unsigned rsel = (unsigned)__popc(m) >> 4;
+          nsel += rsel;
+          if (want_rowlen) {
+#pragma unroll
+            for (int o = 8; o > 0; o >>= 1) rsel += __shfl_xor_sync(0xFFFFFFFFu, rsel, o);
+            if (hl == 0 && rsel) atomicAdd(&rowlen_out[rr.y >> 16], rsel);
+          }
+        }
+        __syncwarp();  // the half-warp's next chunk may touch the same columns; the slot is reused after
+      }
+      if (q + kSlots - 1 < nmine) issue_sparse(warp + (q + kSlots - 1) * kMacWarps, ring_base + so_i);
+      cp_async_commit();
+      so_i = (so_i == kRingLast) ? 0u : so_i + kSlotBytes;
+      so_p = (so_p == kRingLast) ? 0u : so_p + kSlotBytes;
+    }
+    cp_async_wait<0>();
+    __syncthreads();  // the next round's staging overwrites this round's lists
+    q0 += take;
+  }
+
+  // ---- leave tile t: one partial tile per CTA, summed in CTA order by the last to arrive
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    sh.acc[warp][0][8 * lane + 2 * u] += acc2[u].x;
+    sh.acc[warp][0][8 * lane + 2 * u + 1] += acc2[u].y;
+  }
+  __syncthreads();
+  float s = 0.0f;
+  if (threadIdx.x < kTW) {
+#pragma unroll
+    for (int w = 0; w < kMacWarps; ++w) s += sh.acc[w][0][threadIdx.x] + sh.acc[w][1][threadIdx.x];
+  }
+  const int col = t * kTW + threadIdx.x;
+  if (S == 1) {
+    if (threadIdx.x < kTW && col < O) out[col] = s;
+  } else {
+    float* part = part_all + (size_t)t * S * kTW;
+    if (threadIdx.x < kTW) part[(size_t)sl * kTW + threadIdx.x] = s;
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) sh.flag = (atomicAdd(&tilecnt[t], 1u) == (unsigned)(S - 1));
+    __syncthreads();
+    if (sh.flag) {
+      __threadfence();
+      if (threadIdx.x < kTW) {
+        float tot = 0.0f;
+        for (int k = 0; k < S; ++k) tot += __ldcg(&part[(size_t)k * kTW + threadIdx.x]);
+        if (col < O) out[col] = tot;
+      }
+      if (threadIdx.x == 0) tilecnt[t] = 0u;
     }
   }
 

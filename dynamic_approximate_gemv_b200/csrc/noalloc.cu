@@ -47,7 +47,7 @@ inline size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 // per-tile arrival counters, the dispatch tables and the split-K partials.
 size_t scratch_bytes(int T, int G, int S) {
   return 256 + align256((size_t)T * 4) + align256((size_t)G * 4) + align256((size_t)G * T * 32) +
-         align256((size_t)G * kRecPerGroup * 16) + align256((size_t)S * T * kTW * 4);
+         align256((size_t)G * kRecPerGroup * 8) + align256((size_t)S * T * kTW * 4);
 }
 
 // Carves the scratch in the same order as the handle's own workspace.
@@ -64,8 +64,8 @@ WsPtrs carve(char* b, int T, int G) {
   b += align256((size_t)G * 4);
   w.ut = (unsigned char*)b;
   b += align256((size_t)G * T * 32);
-  w.rec = (uint4*)b;
-  b += align256((size_t)G * kRecPerGroup * 16);
+  w.rec = (uint2*)b;
+  b += align256((size_t)G * kRecPerGroup * 8);
   w.part = (float*)b;
   return w;
 }

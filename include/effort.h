@@ -138,8 +138,8 @@ effort_status_t effort_gemv_split(effort_handle_t h, const void* v, effort_dtype
  *     GPU (unordered streams, concurrent host threads) race and give wrong
  *     results; order them on one stream.
  *   Returns EFFORT_ERR_UNSUPPORTED when the handle's geometry needs more than
- *     EFFORT_STATIC_SCRATCH_BYTES of scratch (4096 x 14336 needs about 0.6 MiB,
- *     14336 x 4096 about 1 MiB), and when the device ordinal is 64 or above.
+ *     EFFORT_STATIC_SCRATCH_BYTES of scratch (4096 x 14336 needs about 0.5 MiB,
+ *     14336 x 4096 about 0.6 MiB), and when the device ordinal is 64 or above.
  */
 effort_status_t effort_gemv_static(effort_handle_t h, const void* v, effort_dtype_t v_dtype, float effort,
                                    float* out, float* cutoff_out, uint64_t* count_out, uint32_t* status_out,
