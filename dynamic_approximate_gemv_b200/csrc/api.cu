@@ -85,8 +85,10 @@ effort_status_t make_geometry(int64_t I, int64_t O, Geometry* g) {
   if (S > g->G) S = g->G;
   g->S = S;
   // rows whose surely-used share reaches this fraction are read from the dense
-  // copy (2 B per weight, register accumulation) instead of their buckets
-  double frac = 0.5;
+  // copy (2 B per weight, register accumulation) instead of their buckets; a
+  // dense tile row costs about as many instructions as a quarter of it read
+  // through the buckets, which puts the break-even near 0.3
+  double frac = 0.3;
   if (const char* env = getenv("EFFORT_DENSE_FRACTION")) {
     const double f = atof(env);
     if (f > 0.0 && f <= 1.0) frac = f;

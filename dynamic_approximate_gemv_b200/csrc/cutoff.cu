@@ -22,7 +22,7 @@
 //           used entirely.  The row's exact fp16 threshold tau_i (smallest
 //           magnitude whose product with |v_i| reaches c) turns the product
 //           rule into a magnitude compare.  Rows with k_i * H >= f * n (f the
-//           dense fraction, 1/2 by default) are "dense" (read from the dense
+//           dense fraction, 0.3 by default) are "dense" (read from the dense
 //           copy), other active rows are "sparse" (read from the sorted
 //           buckets), rows whose largest product is below c are off.  Records
 //           {v_i, tau_i, row} of a 32-row group are written sparse rows first,
@@ -44,50 +44,47 @@ struct CutShared {
   unsigned cand_total;
 };
 
-// Inclusive prefix sum over the block (blockDim.x == kCutThreads).
-__device__ __forceinline__ unsigned block_inclusive_scan(unsigned x, unsigned* warp_tot, unsigned& total) {
+// Over a complete histogram of B digits (B a multiple of kCutThreads / 32 ...
+// any B up to 4 * kCutThreads): D = max{d : weight of digits >= d reaches
+// krem}, and the weight still needed inside digit D.  Three block barriers.
+template <int B>
+__device__ void find_crossing(const unsigned* hist, unsigned krem, CutShared& cs, unsigned& digit, unsigned& knew) {
+  constexpr int q = (B + kCutThreads - 1) / kCutThreads;  // digits per thread, highest digits first
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  // thread j owns digits [B - q (j + 1), B - q j): thread 0 the highest
+  const int hi = B - q * (int)threadIdx.x, lo = max(0, hi - q);
+  unsigned local = 0;
+#pragma unroll
+  for (int u = 0; u < q; ++u)
+    if (hi - 1 - u >= lo) local += hist[hi - 1 - u];
+  // inclusive scan over threads in order (= descending digits)
+  unsigned x = local;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const unsigned y = __shfl_up_sync(0xFFFFFFFFu, x, o);
     if (lane >= o) x += y;
   }
-  if (lane == 31) warp_tot[warp] = x;
+  if (lane == 31) cs.warp_tot[warp] = x;
   __syncthreads();
-  if (warp == 0) {
-    unsigned w = warp_tot[lane];
+  // every warp scans the 32 warp totals itself (no second barrier)
+  unsigned wt = cs.warp_tot[lane];
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const unsigned y = __shfl_up_sync(0xFFFFFFFFu, w, o);
-      if (lane >= o) w += y;
-    }
-    warp_tot[lane] = w;  // inclusive over warps
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned y = __shfl_up_sync(0xFFFFFFFFu, wt, o);
+    if (lane >= o) wt += y;
   }
-  __syncthreads();
-  const unsigned before = warp > 0 ? warp_tot[warp - 1] : 0u;
-  total = warp_tot[31];
-  __syncthreads();
-  return x + before;
-}
-
-// Over a complete histogram of B digits: D = max{d : weight of digits >= d
-// reaches krem}; also the weight still needed inside digit D.
-template <int B>
-__device__ void find_crossing(const unsigned* hist, unsigned krem, CutShared& cs, unsigned& digit, unsigned& knew) {
-  constexpr int q = (B + kCutThreads - 1) / kCutThreads;
-  const int lo = threadIdx.x * q, hi = min(B, lo + q);
-  unsigned local = 0;
-  for (int b = lo; b < hi; ++b) local += hist[b];
-  unsigned total;
-  const unsigned incl = block_inclusive_scan(local, cs.warp_tot, total);
-  unsigned cum = total - incl;  // weight of all digits above my range
-  for (int b = hi - 1; b >= lo; --b) {
-    const unsigned nb = hist[b];
-    if (cum < krem && cum + nb >= krem) {
-      cs.sel_digit = (unsigned)b;
-      cs.sel_krem = krem - cum;
+  const unsigned before = __shfl_sync(0xFFFFFFFFu, wt, warp > 0 ? warp - 1 : 0) * (warp > 0 ? 1u : 0u);
+  unsigned cum = before + x - local;  // weight of all digits above this thread's
+  if (cum < krem && cum + local >= krem) {
+    for (int d = hi - 1; d >= lo; --d) {
+      const unsigned nb = hist[d];
+      if (cum + nb >= krem) {
+        cs.sel_digit = (unsigned)d;
+        cs.sel_krem = krem - cum;
+        break;
+      }
+      cum += nb;
     }
-    cum += nb;
   }
   __syncthreads();
   digit = cs.sel_digit;
@@ -238,10 +235,15 @@ __global__ void __launch_bounds__(kCutThreads, 1) k_cutoff_dispatch(const __grid
     for (int b = threadIdx.x; b < kBins0; b += blockDim.x) h0[b] = 0u;
     for (int b = threadIdx.x; b < per; b += blockDim.x) own[b] = 0u;
     __syncthreads();
-    for (int e = threadIdx.x; e < nr * kP; e += blockDim.x) {
-      const int k = e / nr, r = e - k * nr;
+    // chart entry e = k * RP + r (column-major); k from a float reciprocal,
+    // exact for e < 2^16 and RP <= 2^12
+    const int ne = kP * RP;
+    const float rcp_rp = 1.0f / (float)RP;
+    for (int e = threadIdx.x; e < ne; e += blockDim.x) {
+      const int k = __float2int_rd(((float)e + 0.5f) * rcp_rp);
+      const int r = e - k * RP;
       const int wk = s_pw[k];
-      if (wk > 0) atomicAdd(&h0[(chart[(size_t)k * RP + r] >> 19) & (kBins0 - 1)], (unsigned)wk);
+      if (r < nr && wk > 0) atomicAdd(&h0[(chart[e] >> 19) & (kBins0 - 1)], (unsigned)wk);
     }
     cluster.sync();  // every CTA's slice is zeroed and its local histogram complete
     for (int b = threadIdx.x; b < kBins0; b += blockDim.x) {
@@ -268,14 +270,21 @@ __global__ void __launch_bounds__(kCutThreads, 1) k_cutoff_dispatch(const __grid
     prefix = digit << 19;
     pmask = (unsigned)(kBins0 - 1) << 19;
     krem = knew;
-    // ---- this CTA's entries in the chosen bin
-    for (int e = threadIdx.x; e < nr * kP; e += blockDim.x) {
-      const int k = e / nr, r = e - k * nr;
+    // ---- this CTA's entries in the chosen bin (one atomic per warp)
+    for (int e = threadIdx.x; e < ne; e += blockDim.x) {
+      const int k = __float2int_rd(((float)e + 0.5f) * rcp_rp);
+      const int r = e - k * RP;
       const int wk = s_pw[k];
-      const unsigned x = chart[(size_t)k * RP + r];
-      if (wk > 0 && (x & pmask) == prefix) {
-        const unsigned slot = atomicAdd(&cs.ncand, 1u);
-        if (slot < (unsigned)kCandLocal) {
+      const unsigned x = chart[e];
+      const bool in = r < nr && wk > 0 && (x & pmask) == prefix;
+      const unsigned bal = __ballot_sync(0xFFFFFFFFu, in);
+      if (bal) {
+        const int ln = threadIdx.x & 31;
+        unsigned base = 0;
+        if (ln == 0) base = atomicAdd(&cs.ncand, (unsigned)__popc(bal));
+        base = __shfl_sync(0xFFFFFFFFu, base, 0);
+        const unsigned slot = base + (unsigned)__popc(bal & ((1u << ln) - 1u));
+        if (in && slot < (unsigned)kCandLocal) {
           cval[slot] = x;
           cwt[slot] = (unsigned short)wk;
         }
@@ -283,17 +292,19 @@ __global__ void __launch_bounds__(kCutThreads, 1) k_cutoff_dispatch(const __grid
     }
     __syncthreads();
     cluster.sync();  // every list complete; no CTA reads another's merged slice any more
-    if (threadIdx.x == 0) {
-      unsigned tot = 0;
-      bool over = false;
-      for (int r = 0; r < cl; ++r) {
-        const unsigned nc = *cluster.map_shared_rank(&cs.ncand, r);
-        over |= nc > (unsigned)kCandLocal;
-        cs.cand_off[r] = tot;
-        tot += nc;
+    if (threadIdx.x < 32) {  // the cl list lengths, read in parallel, and their offsets
+      const int ln = threadIdx.x;
+      const unsigned nc = (ln < cl) ? *cluster.map_shared_rank(&cs.ncand, ln) : 0u;
+      const bool over = __any_sync(0xFFFFFFFFu, nc > (unsigned)kCandLocal);
+      unsigned incl = nc;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (ln >= o) incl += y;
       }
-      cs.cand_off[cl] = tot;
-      cs.cand_total = over ? 0xFFFFFFFFu : tot;
+      if (ln < cl) cs.cand_off[ln + 1] = incl;
+      if (ln == 0) cs.cand_off[0] = 0u;
+      if (ln == 31) cs.cand_total = over ? 0xFFFFFFFFu : incl;
     }
     __syncthreads();
     const unsigned total = cs.cand_total;

@@ -26,7 +26,14 @@ constexpr int kTW = 256;         // output-tile width (u8 local column)
 constexpr int kCap = 256;        // bucket capacity (entries)
 constexpr int kP = 16;           // probes per row
 constexpr int kCutThreads = 1024;
-constexpr int kMacThreads = 512;
+#ifndef EFFORT_MAC_THREADS
+#define EFFORT_MAC_THREADS 384  // multiply kernel block size
+#endif
+#ifndef EFFORT_MAC_BLOCKS_PER_SM
+#define EFFORT_MAC_BLOCKS_PER_SM 2  // resident multiply blocks per SM the register budget is sized for
+#endif
+constexpr int kMacThreads = EFFORT_MAC_THREADS;
+constexpr int kMacBlocksPerSM = EFFORT_MAC_BLOCKS_PER_SM;
 constexpr int kMacWarps = kMacThreads / 32;
 constexpr int kPrepThreads = 1024;
 constexpr int kDenseThreads = 256;

@@ -41,7 +41,8 @@ constexpr int kSlots = 6;
 constexpr int kSlotBytes = 512;     // one dense tile row, or four chunks
 constexpr int kChunk = 32;          // bucket entries per sparse chunk
 constexpr int kChunkBytes = 128;    // 64 B values, 32 B columns, 32 B unused
-constexpr int kRoundGroups = 32;    // groups staged per round (two per warp)
+constexpr int kRoundGroups = 32;    // groups staged per round
+constexpr int kGroupsPerWarp = (kRoundGroups + kMacWarps - 1) / kMacWarps;
 constexpr int kRoundRows = kRoundGroups * 32;
 constexpr int kMaxChunks = 1280;    // a round takes only the leading groups whose chunks fit
 
@@ -90,10 +91,10 @@ __device__ __forceinline__ unsigned ge_mask(unsigned w2, unsigned tau2) {
 
 
 template <int NJ, bool STATS>
-__global__ void __launch_bounds__(kMacThreads, 2) k_mac(const __grid_constant__ Jobs<NJ> jobs, int S) {
+__global__ void __launch_bounds__(kMacThreads, kMacBlocksPerSM) k_mac(const __grid_constant__ Jobs<NJ> jobs, int S) {
   extern __shared__ __align__(16) unsigned char dyn_smem[];
   MacSmem& sh = *reinterpret_cast<MacSmem*>(dyn_smem);
-  const Job& jb = jobs.j[blockIdx.y];
+  const Job& jb = jobs.j[NJ == 1 ? 0 : blockIdx.y];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   // every field used below is read once from the parameter bank into registers
   const uint16_t* __restrict__ wdense = jb.hd.wdense;
@@ -117,6 +118,10 @@ __global__ void __launch_bounds__(kMacThreads, 2) k_mac(const __grid_constant__ 
 
   // wait for this call's cutoff/dispatch grid (programmatic dependent launch)
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  // the next grid of the stream may launch once every CTA of this one is
+  // resident (each has passed this point); it waits for this grid's completion
+  // before touching what this grid reads or writes
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   const float c = *reinterpret_cast<volatile float*>(jb.ws.c);
   const bool count_all = (__float_as_uint(c) == 0u);
@@ -145,13 +150,13 @@ __global__ void __launch_bounds__(kMacThreads, 2) k_mac(const __grid_constant__ 
 
   for (int q0 = gb; q0 < ge;) {
     const int ng_load = min(kRoundGroups, ge - q0);
-    // ---- stage: warp w reads groups q0 + w and q0 + w + 16 (records, read
+    // ---- stage: warp w reads groups q0 + w, q0 + w + NW, ... (records, read
     // bounds and counts in one round of loads; records past a group's counts
     // are stale and ignored)
-    uint2 rr[2];
-    unsigned uu[2], gc[2];
+    uint2 rr[kGroupsPerWarp];
+    unsigned uu[kGroupsPerWarp], gc[kGroupsPerWarp];
 #pragma unroll
-    for (int z = 0; z < 2; ++z) {
+    for (int z = 0; z < kGroupsPerWarp; ++z) {
       const int gq = warp + kMacWarps * z;
       rr[z] = make_uint2(0, 0);
       uu[z] = gc[z] = 0;
@@ -162,9 +167,9 @@ __global__ void __launch_bounds__(kMacThreads, 2) k_mac(const __grid_constant__ 
         uu[z] = ut[(g * T + t) * 32 + lane];
       }
     }
-    int nck[2], cincl[2];
+    int nck[kGroupsPerWarp], cincl[kGroupsPerWarp];
 #pragma unroll
-    for (int z = 0; z < 2; ++z) {
+    for (int z = 0; z < kGroupsPerWarp; ++z) {
       const int gq = warp + kMacWarps * z;
       const int ns = (int)(gc[z] & 0xFFu), nd = (int)((gc[z] >> 8) & 0xFFu);
       const unsigned U = (uu[z] == 255u) ? (unsigned)kCap : uu[z];
@@ -201,7 +206,7 @@ __global__ void __launch_bounds__(kMacThreads, 2) k_mac(const __grid_constant__ 
     const int NC0 = __shfl_sync(0xFFFFFFFFu, oc, take - 1);  // chunks of the taken groups
     const int NC = (NC0 + 3) & ~3;                            // padded to whole items
 #pragma unroll
-    for (int z = 0; z < 2; ++z) {
+    for (int z = 0; z < kGroupsPerWarp; ++z) {
       const int gq = warp + kMacWarps * z;
       if (gq < take) {  // warp-uniform
         const int src = gq > 0 ? gq - 1 : 0;
