@@ -26,10 +26,10 @@
 //                its own shared copy of the tile.  The entries of one bucket
 //                have distinct columns, so a half-warp updates its copy with
 //                plain loads and stores; a __syncwarp separates its chunks.
-// Each warp streams its items through a ring of 512-byte slots in shared
-// memory filled with cp.async (16 bytes per lane; bytes past a chunk's end are
-// zero-filled by the copy), so several items per warp are in flight without
-// holding registers.  At the end a CTA sums its warp copies and registers into
+// Each warp loads a batch of items straight into registers (16 bytes per lane
+// for a dense tile row, 4 + 2 bytes per lane for a chunk step), so several
+// items per warp are in flight, then works through the batch.  At the end a
+// CTA sums its warp copies and registers into
 // one partial tile; the last of the S CTAs of a tile to arrive adds the
 // partials in slice order (no float atomics: results are reproducible run to
 // run).
@@ -37,14 +37,13 @@
 
 namespace effort {
 
-constexpr int kSlots = 6;
-constexpr int kSlotBytes = 512;     // one dense tile row, or four chunks
 constexpr int kChunk = 32;          // bucket entries per sparse chunk
-constexpr int kChunkBytes = 128;    // 64 B values, 32 B columns, 32 B unused
+constexpr int kDenseBatch = 8;      // dense tile rows a warp has in flight
+constexpr int kSparseBatch = 8;     // chunk steps a warp has in flight
 constexpr int kRoundGroups = 32;    // groups staged per round
 constexpr int kGroupsPerWarp = (kRoundGroups + kMacWarps - 1) / kMacWarps;
 constexpr int kRoundRows = kRoundGroups * 32;
-constexpr int kMaxChunks = 1280;    // a round takes only the leading groups whose chunks fit
+constexpr int kMaxChunks = 2048;    // a round takes only the leading groups whose chunks fit
 
 // Staged work of one round:
 //   dense row  {v bits, tau | row << 16}
@@ -57,11 +56,9 @@ struct MacSmem {
   int gtot[2][kRoundGroups];     // per staged group: dense rows, chunks
   unsigned long long warp_cnt[kMacWarps];
   int flag;
-  alignas(16) unsigned char ring[kMacWarps][kSlots][kSlotBytes];
 };
 
-__device__ __forceinline__ unsigned smem_u32(const void* p) { return (unsigned)__cvta_generic_to_shared(p); }
-// Streamed weights are read once per call: they are copied with an L2
+// Streamed weights are read once per call: they bypass L1 and carry an L2
 // evict-first policy so that they do not push the kernels' code, the dispatch
 // records and the tables out of L2.
 __device__ __forceinline__ unsigned long long evict_first_policy() {
@@ -69,19 +66,22 @@ __device__ __forceinline__ unsigned long long evict_first_policy() {
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
   return p;
 }
-__device__ __forceinline__ void cp_async16(unsigned dst, const void* gsrc, unsigned long long pol) {
-  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, 16, %2;\n" ::"r"(dst), "l"(gsrc), "l"(pol)
-               : "memory");
+__device__ __forceinline__ uint4 ld_stream_v4(const void* p, unsigned long long pol) {
+  uint4 x;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+               : "=r"(x.x), "=r"(x.y), "=r"(x.z), "=r"(x.w)
+               : "l"(p), "l"(pol));
+  return x;
 }
-// copies `bytes` (0..16) and zero-fills the rest of the 16-byte destination
-__device__ __forceinline__ void cp_async16_zfill(unsigned dst, const void* gsrc, unsigned bytes, unsigned long long pol) {
-  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;\n" ::"r"(dst), "l"(gsrc), "r"(bytes),
-               "l"(pol) : "memory");
+__device__ __forceinline__ unsigned ld_stream_u32(const void* p, unsigned long long pol) {
+  unsigned x;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.u32 %0, [%1], %2;" : "=r"(x) : "l"(p), "l"(pol));
+  return x;
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+__device__ __forceinline__ unsigned ld_stream_u16(const void* p, unsigned long long pol) {
+  unsigned short x;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.u16 %0, [%1], %2;" : "=h"(x) : "l"(p), "l"(pol));
+  return x;
 }
 // mask with 0xFFFF in each half whose magnitude is >= tau (both halves hold tau)
 __device__ __forceinline__ unsigned ge_mask(unsigned w2, unsigned tau2) {
@@ -130,23 +130,9 @@ __global__ void __launch_bounds__(kMacThreads, kMacBlocksPerSM) k_mac(const __gr
 #pragma unroll
   for (int u = 0; u < 4; ++u) acc2[u] = make_float2(0.0f, 0.0f);
   unsigned nsel = 0;
-  unsigned char* ring = sh.ring[warp][0];
-  const unsigned ring_base = smem_u32(ring);
   const unsigned long long pol = evict_first_policy();
   const int h = lane >> 4, hl = lane & 15;
   float* acc_h = sh.acc[warp][h];
-  // copy roles for a sparse item: chunk cp_ck = lane / 6 (lanes 0..23); four
-  // lanes copy its 64 value bytes, two lanes its 32 column bytes
-  const int cp_ck = lane / 6, cp_r = lane - 6 * (lane / 6);
-  const bool cp_val = cp_r < 4;
-  const int cp_sub = cp_val ? cp_r : cp_r - 4;
-  const bool cp_act = lane < 24;
-  const unsigned cp_dst = (unsigned)(kChunkBytes * cp_ck + (cp_val ? 16 * cp_sub : 64 + 16 * cp_sub));
-  // source of lane's 16 bytes: base + first * mul, valid bytes len * mul - 16 sub
-  const char* cp_base = cp_val ? reinterpret_cast<const char*>(vals) + 16 * cp_sub
-                               : reinterpret_cast<const char*>(idxs) + 16 * cp_sub;
-  const unsigned cp_mul = cp_val ? 2u : 1u;
-  const int cp_off = 16 * cp_sub;
 
   for (int q0 = gb; q0 < ge;) {
     const int ng_load = min(kRoundGroups, ge - q0);
@@ -226,90 +212,80 @@ __global__ void __launch_bounds__(kMacThreads, kMacBlocksPerSM) k_mac(const __gr
     }
     if (threadIdx.x < NC - NC0) sh.chunk[NC0 + threadIdx.x] = make_uint4(0u, 0u, 0u, 0x7C00u);
     __syncthreads();
-    const int NI = ND + NC / 4;  // dense rows, then items of four chunks
-    // this warp's items: j = warp + 16 q; dense while q < nmineD
-    const int nmine = (NI > warp) ? (NI - warp + kMacWarps - 1) / kMacWarps : 0;
-    const int nmineD = (ND > warp) ? (ND - warp + kMacWarps - 1) / kMacWarps : 0;
-
-    // sparse item j: lanes 0..23 copy their 16 bytes of chunk 4 (j - ND) + cp_ck
-    auto issue_sparse = [&](int j, unsigned dst) {
-      if (cp_act) {
-        const uint2 r = *reinterpret_cast<const uint2*>(&sh.chunk[4 * (j - ND) + cp_ck]);  // {first, entries}
-        const int nb = min(16, max(0, (int)(r.y * cp_mul) - cp_off));
-        cp_async16_zfill(dst + cp_dst, cp_base + (size_t)r.x * cp_mul, (unsigned)nb, pol);
-      }
-    };
-    auto issue = [&](int q, unsigned dst) {  // the warp's q-th item into the ring slot at dst
-      const int j = warp + q * kMacWarps;
-      if (q < nmineD) {
-        const unsigned row = sh.recD[j].y >> 16;
-        cp_async16(dst + 16 * lane, wdense + (size_t)row * dstride + (size_t)t * kTW + 8 * lane, pol);
-      } else if (q < nmine) {
-        issue_sparse(j, dst);
-      }
-      cp_async_commit();
-    };
-    constexpr unsigned kRingLast = (kSlots - 1) * kSlotBytes;
-    unsigned so_i = 0, so_p = 0;  // byte offsets of the next slot to fill and to process
+    // ---- dense rows: warp w takes rows j = w, w + NW, ... in batches, each
+    // lane reading 16 bytes (8 columns) of every row's tile
+    for (int j0 = warp; j0 < ND; j0 += kDenseBatch * kMacWarps) {
+      uint4 wv[kDenseBatch];
+      uint2 rd[kDenseBatch];
 #pragma unroll
-    for (int q = 0; q < kSlots - 1; ++q) {
-      issue(q, ring_base + so_i);
-      so_i = (so_i == kRingLast) ? 0u : so_i + kSlotBytes;
-    }
-    int q = 0;
-    // dense items: 8 columns per lane, accumulated in registers
-    for (; q < nmineD; ++q) {
-      cp_async_wait<kSlots - 2>();
-      __syncwarp();
-      const uint2 r = sh.recD[warp + q * kMacWarps];
-      const float vi = __uint_as_float(r.x);
-      const unsigned tau2 = (r.y & 0xFFFFu) * 0x10001u;
-      const uint4 wv = *reinterpret_cast<const uint4*>(ring + so_p + 16 * lane);
-      const unsigned wr[4] = {wv.x, wv.y, wv.z, wv.w};
-      const float2 v2 = make_float2(vi, vi);
-      unsigned rsel = 0;
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const unsigned m = ge_mask(wr[u], tau2);
-        const unsigned wk = wr[u] & m;  // unused weights become +0
-        acc2[u] = __ffma2_rn(v2, __half22float2(*reinterpret_cast<const __half2*>(&wk)), acc2[u]);
-        if (STATS) rsel += (unsigned)__popc(m) >> 4;
-      }
-      if (STATS) {
-        nsel += rsel;
-        if (want_rowlen) {
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) rsel += __shfl_xor_sync(0xFFFFFFFFu, rsel, o);
-          if (lane == 0 && rsel) atomicAdd(&rowlen_out[r.y >> 16], rsel);
+      for (int u = 0; u < kDenseBatch; ++u) {
+        const int j = j0 + u * kMacWarps;
+        rd[u] = make_uint2(0u, 0x7C00u);  // past the list: tau = +inf, nothing passes
+        wv[u] = make_uint4(0u, 0u, 0u, 0u);
+        if (j < ND) {
+          rd[u] = sh.recD[j];
+          wv[u] = ld_stream_v4(wdense + (size_t)(rd[u].y >> 16) * dstride + (size_t)t * kTW + 8 * lane, pol);
         }
       }
-      __syncwarp();  // the slot is free for the next copy
-      issue(q + kSlots - 1, ring_base + so_i);
-      so_i = (so_i == kRingLast) ? 0u : so_i + kSlotBytes;
-      so_p = (so_p == kRingLast) ? 0u : so_p + kSlotBytes;
-    }
-    // sparse items: half-warp h takes chunks 2h and 2h + 1 of the item in turn,
-    // 2 entries per lane
-    for (; q < nmine; ++q) {
-      cp_async_wait<kSlots - 2>();
-      __syncwarp();
-      const int cb0 = 4 * (warp + q * kMacWarps - ND) + 2 * h;
 #pragma unroll
-      for (int kk = 0; kk < 2; ++kk) {
-        const uint2 rr = *reinterpret_cast<const uint2*>(&sh.chunk[cb0 + kk].z);  // {v bits, tau | row << 16}
-        const unsigned char* cb = ring + so_p + kChunkBytes * (2 * h + kk);
-        const float vi = __uint_as_float(rr.x);
-        const unsigned tau2 = (rr.y & 0xFFFFu) * 0x10001u;
-        const unsigned w2 = *reinterpret_cast<const unsigned*>(cb + 4 * hl);
-        const unsigned ix = *reinterpret_cast<const unsigned short*>(cb + 64 + 2 * hl);
-        const unsigned m = ge_mask(w2, tau2);  // zero-filled entries have w = 0 < tau
-        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w2));
+      for (int u = 0; u < kDenseBatch; ++u) {
+        const float vi = __uint_as_float(rd[u].x);
+        const unsigned tau2 = (rd[u].y & 0xFFFFu) * 0x10001u;
+        const unsigned wr[4] = {wv[u].x, wv[u].y, wv[u].z, wv[u].w};
+        const float2 v2 = make_float2(vi, vi);
+        unsigned rsel = 0;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const unsigned m = ge_mask(wr[k], tau2);
+          const unsigned wk = wr[k] & m;  // unused weights become +0
+          acc2[k] = __ffma2_rn(v2, __half22float2(*reinterpret_cast<const __half2*>(&wk)), acc2[k]);
+          if (STATS) rsel += (unsigned)__popc(m) >> 4;
+        }
+        if (STATS) {
+          nsel += rsel;
+          if (want_rowlen) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) rsel += __shfl_xor_sync(0xFFFFFFFFu, rsel, o);
+            if (lane == 0 && rsel) atomicAdd(&rowlen_out[rd[u].y >> 16], rsel);
+          }
+        }
+      }
+    }
+    // ---- sparse chunks: step s takes chunk 2s for half-warp 0 and 2s + 1 for
+    // half-warp 1; each lane reads 2 entries (values and columns) of its chunk
+    const int NS = NC / 2;
+    for (int s0 = warp; s0 < NS; s0 += kSparseBatch * kMacWarps) {
+      unsigned w2[kSparseBatch], ix[kSparseBatch];
+      uint2 vr[kSparseBatch];  // {v bits, tau | row << 16}
+#pragma unroll
+      for (int u = 0; u < kSparseBatch; ++u) {
+        const int st = s0 + u * kMacWarps;
+        w2[u] = 0u;
+        ix[u] = 0u;
+        vr[u] = make_uint2(0u, 0x7C00u);
+        if (st < NS) {
+          const uint4 cr = sh.chunk[2 * st + h];  // {first entry, entries, v bits, tau | row << 16}
+          vr[u] = make_uint2(cr.z, cr.w);
+          // entries past the chunk are not read; the odd one that shares a
+          // lane's 4 bytes lies past the read bound, so its |w| < tau
+          if (2 * hl < (int)cr.y) {
+            w2[u] = ld_stream_u32(vals + cr.x + 2 * hl, pol);
+            ix[u] = ld_stream_u16(idxs + cr.x + 2 * hl, pol);
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kSparseBatch; ++u) {
+        const float vi = __uint_as_float(vr[u].x);
+        const unsigned tau2 = (vr[u].y & 0xFFFFu) * 0x10001u;
+        const unsigned m = ge_mask(w2[u], tau2);
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w2[u]));
         if (m & 0xFFFFu) {
-          float* a = acc_h + (ix & 0xFFu);
+          float* a = acc_h + (ix[u] & 0xFFu);
           *a = fmaf(vi, f.x, *a);
         }
         if (m >> 16) {
-          float* a = acc_h + (ix >> 8);
+          float* a = acc_h + (ix[u] >> 8);
           *a = fmaf(vi, f.y, *a);
         }
         if (STATS) {
@@ -318,17 +294,12 @@ __global__ void __launch_bounds__(kMacThreads, kMacBlocksPerSM) k_mac(const __gr
           if (want_rowlen) {
 #pragma unroll
             for (int o = 8; o > 0; o >>= 1) rsel += __shfl_xor_sync(0xFFFFFFFFu, rsel, o);
-            if (hl == 0 && rsel) atomicAdd(&rowlen_out[rr.y >> 16], rsel);
+            if (hl == 0 && rsel) atomicAdd(&rowlen_out[vr[u].y >> 16], rsel);
           }
         }
-        __syncwarp();  // the half-warp's next chunk may touch the same columns; the slot is reused after
+        __syncwarp();  // the half-warp's next chunk may touch the same columns
       }
-      if (q + kSlots - 1 < nmine) issue_sparse(warp + (q + kSlots - 1) * kMacWarps, ring_base + so_i);
-      cp_async_commit();
-      so_i = (so_i == kRingLast) ? 0u : so_i + kSlotBytes;
-      so_p = (so_p == kRingLast) ? 0u : so_p + kSlotBytes;
     }
-    cp_async_wait<0>();
     __syncthreads();  // the next round's staging overwrites this round's lists
     q0 += take;
   }
