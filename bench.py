@@ -324,32 +324,41 @@ def main():
     us_per_step = ms * 1000.0 / a.steps
     value = us_per_step / world  # whole job: all ranks' matvecs over the max-rank time
 
-    # per-kernel durations (events between the two kernels), same rotation and effort
+    # per-kernel durations: the split call records an event between the two
+    # kernels; the calls are captured in a CUDA graph (external event-record
+    # nodes) so that host launch gaps do not enter the kernel times
     n_ph = GRAPH_STEPS
     s = torch.cuda.Stream(device=dev)
-    evA = [torch.cuda.Event(enable_timing=True) for _ in range(n_ph + 1)]
-    evB = [torch.cuda.Event(enable_timing=True) for _ in range(n_ph)]
-    for ev in evB:
-        ev.record(s)  # creates the CUDA events the library records into
+    evA = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n_ph + 1)]
+    evB = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n_ph)]
+    for ev in evA + evB:
+        ev.record(s)  # creates the CUDA events
     torch.cuda.synchronize()
 
-    def phase_pass():
-        with torch.cuda.stream(s):
-            for k, (mi, vi) in enumerate(step_pairs(n_ph)):
-                evA[k].record(s)
-                mats[mi].gemv_split(vecs[vi], EFFORT, outs[mi], evB[k], stream=s)
-            evA[n_ph].record(s)
-        torch.cuda.synchronize()
+    def phase_calls():
+        for k, (mi, vi) in enumerate(step_pairs(n_ph)):
+            evA[k].record(s)
+            mats[mi].gemv_split(vecs[vi], EFFORT, outs[mi], evB[k], stream=s)
+        evA[n_ph].record(s)
 
-    for _ in range(3):
-        phase_pass()
+    s.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(s):
+        phase_calls()  # warm once outside capture
+    torch.cuda.synchronize()
+    gph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gph, stream=s):
+        phase_calls()
+    torch.cuda.synchronize()
     cut_ms, mac_ms = [], []
-    for _ in range(5):
-        phase_pass()
-        cut_ms += [evA[k].elapsed_time(evB[k]) for k in range(n_ph)]
-        mac_ms += [evB[k].elapsed_time(evA[k + 1]) for k in range(n_ph)]
+    for rep in range(8):
+        gph.replay()
+        torch.cuda.synchronize()
+        if rep >= 3:
+            cut_ms += [evA[k].elapsed_time(evB[k]) for k in range(n_ph)]
+            mac_ms += [evB[k].elapsed_time(evA[k + 1]) for k in range(n_ph)]
     mac_us = statistics.mean(mac_ms) * 1000.0
     cut_us = statistics.mean(cut_ms) * 1000.0
+    del gph
 
     S_mean = mean_count(EFFORT)
     alg_bytes = 3.0 * S_mean + 4.0 * IN_DIM + 4.0 * OUT_DIM  # F3 bytes of the used set + v + out

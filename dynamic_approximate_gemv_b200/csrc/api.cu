@@ -359,7 +359,16 @@ effort_status_t effort_gemv_split(effort_handle_t h, const void* v, effort_dtype
   cudaStream_t s = (cudaStream_t)stream;
   h->last_stream = s;
   cudaError_t e = launch_cutoff(jobs, h->g.I, h->g.cl, s);
-  if (e == cudaSuccess) e = cudaEventRecord((cudaEvent_t)mid_event, s);
+  // under stream capture the event is recorded as an external event-record
+  // node, so that the phases of a captured graph can be timed too
+  if (e == cudaSuccess) {
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    e = cudaStreamIsCapturing(s, &cap);
+    if (e == cudaSuccess)
+      e = (cap == cudaStreamCaptureStatusActive)
+              ? cudaEventRecordWithFlags((cudaEvent_t)mid_event, s, cudaEventRecordExternal)
+              : cudaEventRecord((cudaEvent_t)mid_event, s);
+  }
   if (e == cudaSuccess) e = launch_mac(jobs, h->g.T, h->g.S, s);
   if (e != cudaSuccess) {
     cudaGetLastError();

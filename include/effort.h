@@ -109,6 +109,8 @@ effort_status_t effort_gemv_ex(effort_handle_t h, const void* v, effort_dtype_t 
  *   the cutoff/dispatch kernel and the multiply kernel, so that each phase can
  *   be timed with events.  The multiply kernel then starts after the event
  *   instead of launching early against the first kernel.  mid_event non-NULL.
+ *   Under stream capture the event is recorded with cudaEventRecordExternal,
+ *   so that it becomes an event-record node of the CUDA graph.
  */
 effort_status_t effort_gemv_split(effort_handle_t h, const void* v, effort_dtype_t v_dtype, float effort,
                                   float* out, float* cutoff_out, uint64_t* count_out, void* mid_event,
