@@ -116,6 +116,30 @@ def run_reference(a):
     print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------- ranks
+def replica_seed(rank, m):
+    """Seed of prepared matrix m on `rank`: each rank runs its own replica
+    (the path does not shard; there is no data-path collective)."""
+    return 1000 * (rank + 1) + m
+
+
+def max_over_ranks(x, world, device):
+    """The largest of the ranks' values (timing is the slowest rank's)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_us_per_matvec(us_per_step_max, world):
+    """Whole-job figure: every rank did one matvec per step, so the job did
+    `world` matvecs in the slowest rank's step time."""
+    return us_per_step_max / world
+
+
 # ----------------------------------------------------------------- clocks
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -241,17 +265,13 @@ def main():
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def rank_max(x):
+        return max_over_ranks(x, world, dev)
 
     g = torch.Generator(device=dev)
     mats, raws = [], []
     for m in range(N_MATS):
-        g.manual_seed(1000 * (rank + 1) + m)
+        g.manual_seed(replica_seed(rank, m))
         W = (torch.randn(IN_DIM, OUT_DIM, device=dev, generator=g) * 0.02).to(torch.float16)
         mats.append(E.PreparedMatrix(W, KEEP))
         raws.append(W)
@@ -305,7 +325,7 @@ def main():
         e1.record()
         torch.cuda.synchronize()
         barrier()
-        ms = max_over_ranks(e0.elapsed_time(e1))
+        ms = rank_max(e0.elapsed_time(e1))
         # keep the same replay running until the clock sampler has a window of samples
         if sampler is not None and min_seconds > 0:
             t0 = time.perf_counter()
@@ -322,7 +342,7 @@ def main():
     ms = timed_steps(EFFORT, a.steps, a.warmup, sampler, min_seconds=2.0)
     clocks = sampler.stop()
     us_per_step = ms * 1000.0 / a.steps
-    value = us_per_step / world  # whole job: all ranks' matvecs over the max-rank time
+    value = whole_job_us_per_matvec(us_per_step, world)
 
     # per-kernel durations: the split call records an event between the two
     # kernels; the calls are captured in a CUDA graph (external event-record
@@ -441,7 +461,7 @@ def main():
     e1.record()
     torch.cuda.synchronize()
     barrier()
-    e2e_us = max_over_ranks(e0.elapsed_time(e1)) * 1000.0 / n_e2e / world
+    e2e_us = rank_max(e0.elapsed_time(e1)) * 1000.0 / n_e2e / world
 
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
