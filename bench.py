@@ -441,6 +441,36 @@ def main():
             sweep[str(e)] = {"us": us, "gbs_algorithmic": b / (us * 1e-6) / 1e9, "mean_used": Se,
                              "vs_dense_roofline_measured": baselines["dense_roofline_us_measured_peak"] / us}
 
+    # batched / MoE: 8 experts of the workload's shape (the first eight prepared
+    # matrices), n vectors N(0,1) each routed to its top-2 experts by a seeded
+    # N(0,1)/64 gate (ties to the lower expert), one cutoff per (vector, expert)
+    # pair, all pairs in one batched call
+    moe = {}
+    if not a.no_sweep:
+        n_exp = 8
+        gate = inputs.gate(n_exp, IN_DIM, 300)
+        ws_moe = E.Workspace(IN_DIM, OUT_DIM, max_pairs=32)
+        for nv in (1, 4, 16):
+            Vn = np.stack([inputs.vector(IN_DIM, 200 + 16 * nv + k) for k in range(nv)])
+            order = np.argsort(-(gate.astype(np.float64) @ Vn.astype(np.float64).T), axis=0, kind="stable")
+            hidx = [int(order[r, k]) for k in range(nv) for r in range(2)]
+            vidx = [k for k in range(nv) for _ in range(2)]
+            Vd = torch.from_numpy(Vn).to(dev)
+            OUTd = torch.empty(2 * nv, OUT_DIM, device=dev)
+            cnt_d = torch.zeros(2 * nv, device=dev, dtype=torch.int64)
+            row = {}
+            for e in (0.5, 0.25, 0.12):
+                E.gemv_batched(ws_moe, mats[:n_exp], hidx, vidx, Vd, [e] * (2 * nv), OUT=OUTd, counts=cnt_d)
+                torch.cuda.synchronize()
+                used = float(cnt_d.sum().item())
+                ms_call = time_graph(lambda: E.gemv_batched(ws_moe, mats[:n_exp], hidx, vidx, Vd, [e] * (2 * nv),
+                                                            OUT=OUTd), n_rep=20)
+                b = 3.0 * used + 2 * nv * (4.0 * IN_DIM + 4.0 * OUT_DIM)
+                row[str(e)] = {"us_per_call": ms_call * 1000.0, "pairs": 2 * nv,
+                               "gbs_algorithmic": b / (ms_call * 1e-3) / 1e9}
+            moe[str(nv)] = row
+        ws_moe.close()
+
     # end to end through the public API: pinned host v -> device, gemv, out -> pinned host
     n_e2e = min(a.steps, 400)
     hv = [torch.from_numpy(inputs.vector(IN_DIM, 7 + k, "t3")).pin_memory() for k in range(N_VECS)]
@@ -479,7 +509,9 @@ def main():
                         "d2h_bytes_per_step": 4 * OUT_DIM},
                 "gpu_launches": 2 * a.steps, "clocks": clocks,
                 "phases_us": {"cutoff_dispatch": cut_us, "mac": mac_us},
-                "mean_used_products": S_mean, "baselines": baselines, "sweep": sweep}
+                "mean_used_products": S_mean, "baselines": baselines, "sweep": sweep,
+                "moe": {"workload": "8 experts 4096x14336 fp16, n vectors N(0,1) routed top-2 by a seeded gate, "
+                                    "one cutoff per pair, one batched call", "by_n_vectors": moe}}
         print(json.dumps(line), flush=True)
     for m in mats:
         m.close()
