@@ -116,6 +116,137 @@ def run_reference(a):
     print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------- other shapes
+def measure_shape(E, dev, in_dim, out_dim, efforts, dist, n_mats=10, n_vecs=8, seed0=5000, keep=1.0):
+    """us per matvec and algorithmic GB/s on another workload shape: n_mats
+    prepared matrices N(0, 0.02^2) fp16 and n_vecs vectors rotated through CUDA
+    graphs of 40 steps (inputs larger than L2), as for the headline workload."""
+    import torch
+    from dynamic_approximate_gemv_b200 import inputs
+    g = torch.Generator(device=dev)
+    mats = []
+    for m in range(n_mats):
+        g.manual_seed(seed0 + m)
+        W = (torch.randn(in_dim, out_dim, device=dev, generator=g) * 0.02).to(torch.float16)
+        mats.append(E.PreparedMatrix(W, keep))
+        del W
+    vecs = [torch.from_numpy(inputs.vector(in_dim, seed0 + 100 + k, dist)).to(dev) for k in range(n_vecs)]
+    outs = [torch.empty(out_dim, device=dev) for _ in range(n_mats)]
+    cnt = torch.zeros(1, device=dev, dtype=torch.int64)
+    res = {}
+    steps = 40
+    for e in efforts:
+        used = 0.0
+        for k in range(steps):
+            mats[k % n_mats].gemv(vecs[k % n_vecs], e, out=outs[k % n_mats], count=cnt)
+            used += float(cnt.item())
+        used /= steps
+        s = torch.cuda.Stream(device=dev)
+        s.wait_stream(torch.cuda.current_stream(dev))
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(s):
+            for k in range(steps):
+                mats[k % n_mats].gemv(vecs[k % n_vecs], e, out=outs[k % n_mats])
+        torch.cuda.synchronize()
+        with torch.cuda.graph(gr, stream=s):
+            for k in range(steps):
+                mats[k % n_mats].gemv(vecs[k % n_vecs], e, out=outs[k % n_mats])
+        for _ in range(3):
+            gr.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 10
+        e0.record()
+        for _ in range(reps):
+            gr.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) * 1000.0 / (reps * steps)
+        b = 3.0 * used + 4.0 * in_dim + 4.0 * out_dim
+        dense_b = 2.0 * in_dim * out_dim + 4.0 * in_dim + 4.0 * out_dim
+        res[str(e)] = {"us": us, "gbs_algorithmic": b / (us * 1e-6) / 1e9, "mean_used": used,
+                       "dense_roofline_us_measured_peak": dense_b / (hbm_peak()[0] * 1e9) * 1e6}
+        del gr
+    for m in mats:
+        m.close()
+    return res
+
+
+# ----------------------------------------------------------------- decode chain
+CHAIN_MATS = (("q", 0, 0), ("k", 0, 1), ("v", 0, 1), ("o", 0, 0), ("w1", 0, 2), ("w3", 0, 2), ("w2", 2, 0))
+
+
+def rms_norm(y, eps=1e-5):
+    """y / sqrt(mean(y^2) + eps), no gain (harness between matvecs)."""
+    import torch
+    return y * torch.rsqrt(torch.mean(y * y) + eps)
+
+
+def chain_token(E, mats, x, effort):
+    """One token through the stack: per layer x -> q, k, v; q -> o; o -> w1, w3;
+    w1 * w3 -> w2; every matvec input RMS-normalised (no gain)."""
+    for L in mats:
+        xn = rms_norm(x)
+        q = L["q"].gemv(xn, effort)
+        L["k"].gemv(xn, effort)
+        L["v"].gemv(xn, effort)
+        o = L["o"].gemv(rms_norm(q), effort)
+        h = rms_norm(o)
+        a = L["w1"].gemv(h, effort)
+        b = L["w3"].gemv(h, effort)
+        x = rms_norm(L["w2"].gemv(rms_norm(a * b), effort))
+    return x
+
+
+def measure_chain(E, dev, layers=32, dims=(4096, 1024, 14336), effort=0.25, keep=0.8):
+    """Decode stack of Mistral-7B shapes (random init): one token = 7 * layers
+    dependent matvecs, timed as one CUDA graph replay per token."""
+    import torch
+    from dynamic_approximate_gemv_b200 import inputs
+    g = torch.Generator(device=dev)
+    mats, dense_bytes = [], 0.0
+    for l in range(layers):
+        L = {}
+        for m, (name, a, b) in enumerate(CHAIN_MATS):
+            g.manual_seed(1000 * l + m)
+            W = (torch.randn(dims[a], dims[b], device=dev, generator=g) * 0.02).to(torch.float16)
+            L[name] = E.PreparedMatrix(W, keep)
+            dense_bytes += 2.0 * dims[a] * dims[b] + 4.0 * (dims[a] + dims[b])
+            del W
+        mats.append(L)
+    x0 = torch.from_numpy(inputs.vector(dims[0], 9)).to(dev)
+    s = torch.cuda.Stream(device=dev)
+    s.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(s):
+        chain_token(E, mats, x0, effort)
+    torch.cuda.synchronize()
+    gr = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gr, stream=s):
+        chain_token(E, mats, x0, effort)
+    for _ in range(3):
+        gr.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = 10
+    e0.record()
+    for _ in range(reps):
+        gr.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1000.0 / reps
+    storage = sum(L[n].info()["device_bytes"] for L in mats for n in L) if hasattr(mats[0]["q"], "info") else None
+    del gr
+    for L in mats:
+        for n in L:
+            L[n].close()
+    return {"workload": f"{layers} layers of q {dims[0]}x{dims[0]}, k/v {dims[0]}x{dims[1]}, o {dims[0]}x{dims[0]}, "
+                        f"w1/w3 {dims[0]}x{dims[2]}, w2 {dims[2]}x{dims[0]} fp16 N(0,0.02^2), keep {keep}, "
+                        f"effort {effort}; {7 * layers} dependent matvecs per token, RMS-normalised inputs",
+            "us_per_token": us, "matvecs_per_token": 7 * layers, "us_per_matvec": us / (7 * layers),
+            "dense_roofline_us_per_token_measured_peak": dense_bytes / (hbm_peak()[0] * 1e9) * 1e6,
+            "prepared_bytes": storage}
+
+
 # ----------------------------------------------------------------- ranks
 def replica_seed(rank, m):
     """Seed of prepared matrix m on `rank`: each rank runs its own replica
@@ -471,6 +602,17 @@ def main():
             moe[str(nv)] = row
         ws_moe.close()
 
+    # the other shapes of the method's workloads
+    shapes = {}
+    if not a.no_sweep:
+        shapes["attention 4096x4096, v N(0,1)"] = measure_shape(E, dev, 4096, 4096, SWEEP, "normal")
+        shapes["FFN down 14336x4096, v t3/sqrt(3)"] = measure_shape(E, dev, 14336, 4096, (0.25, 0.15), "t3")
+        shapes["FFN up 4096x14336, keep 0.75, v t3/sqrt(3)"] = measure_shape(E, dev, 4096, 14336, (0.25, 0.15),
+                                                                             "t3", keep=0.75)
+
+    # the decode chain (one token through 32 layers)
+    chain = measure_chain(E, dev) if (not a.no_sweep and world == 1) else {}
+
     # end to end through the public API: pinned host v -> device, gemv, out -> pinned host
     n_e2e = min(a.steps, 400)
     hv = [torch.from_numpy(inputs.vector(IN_DIM, 7 + k, "t3")).pin_memory() for k in range(N_VECS)]
@@ -510,6 +652,8 @@ def main():
                 "gpu_launches": 2 * a.steps, "clocks": clocks,
                 "phases_us": {"cutoff_dispatch": cut_us, "mac": mac_us},
                 "mean_used_products": S_mean, "baselines": baselines, "sweep": sweep,
+                "shapes": shapes,
+                "chain": chain,
                 "moe": {"workload": "8 experts 4096x14336 fp16, n vectors N(0,1) routed top-2 by a seeded gate, "
                                     "one cutoff per pair, one batched call", "by_n_vectors": moe}}
         print(json.dumps(line), flush=True)

@@ -1,0 +1,87 @@
+"""A decode chain through the library, checked matvec by matvec (teacher forced).
+
+The stack follows the Mistral-7B layer pattern at a reduced width: per layer
+q, k, v, o, w1, w3, w2 with every matvec input RMS-normalised, each output
+feeding the next step.  Every matvec of two layers is compared with the oracle
+on the GPU's own input to that step: the cutoff bit for bit, the used count
+exactly, the output within the parity tolerance.  Selection exactness is thus
+defined at every step even though the chain's inputs come from the GPU.
+"""
+import os
+import sys
+
+import numpy as np
+import pytest
+import torch
+
+from dynamic_approximate_gemv_b200 import inputs
+from oracle import effort_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+REL_L2 = 1e-4
+MAX_ABS = 1e-3
+
+
+@pytest.fixture(scope="module")
+def E():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from dynamic_approximate_gemv_b200 import build
+    build.build()
+    import dynamic_approximate_gemv_b200 as E
+    E.lib()
+    return E
+
+
+def f32bits(x):
+    return int(np.array([x], np.float32).view(np.uint32)[0])
+
+
+def checked_gemv(pm, prep, x, effort):
+    cutoff = torch.empty(1, device="cuda", dtype=torch.float32)
+    count = torch.full((1,), -1, device="cuda", dtype=torch.int64)
+    out = pm.gemv(x, effort, cutoff=cutoff, count=count)
+    torch.cuda.synchronize()
+    ref = O.effort_gemv(prep, x.cpu().numpy(), effort)
+    assert f32bits(cutoff.item()) == f32bits(ref.c)
+    assert int(count.item()) == ref.count
+    got = out.cpu().numpy().astype(np.float64)
+    nref = np.linalg.norm(ref.out)
+    assert np.linalg.norm(got - ref.out) <= REL_L2 * nref
+    assert np.max(np.abs(got - ref.out)) <= MAX_ABS * np.max(np.abs(ref.out))
+    return out
+
+
+def test_chain_two_layers_teacher_forced(E):
+    sys.path.insert(0, ROOT)
+    import bench
+    dims = (512, 128, 1792)  # d_model, kv width, ffn width (Mistral-7B pattern, scaled by 1/8)
+    layers, effort, keep = 2, 0.25, 0.8
+    mats, preps = [], []
+    for l in range(layers):
+        L, P = {}, {}
+        for m, (name, a, b) in enumerate(bench.CHAIN_MATS):
+            Wn = inputs.weights(dims[a], dims[b], 1000 * l + m)
+            L[name] = E.PreparedMatrix(torch.from_numpy(Wn).cuda(), keep)
+            P[name] = O.Prepared(Wn.view(np.uint16), keep)
+        mats.append(L)
+        preps.append(P)
+    try:
+        x = torch.from_numpy(inputs.vector(dims[0], 9)).cuda()
+        for L, P in zip(mats, preps):
+            xn = bench.rms_norm(x)
+            q = checked_gemv(L["q"], P["q"], xn, effort)
+            checked_gemv(L["k"], P["k"], xn, effort)
+            checked_gemv(L["v"], P["v"], xn, effort)
+            o = checked_gemv(L["o"], P["o"], bench.rms_norm(q), effort)
+            h = bench.rms_norm(o)
+            a = checked_gemv(L["w1"], P["w1"], h, effort)
+            b = checked_gemv(L["w3"], P["w3"], h, effort)
+            x = bench.rms_norm(checked_gemv(L["w2"], P["w2"], bench.rms_norm(a * b), effort))
+        assert torch.isfinite(x).all()
+    finally:
+        for L in mats:
+            for pm in L.values():
+                pm.close()
