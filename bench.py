@@ -70,20 +70,21 @@ def workload_config():
 
 
 # ----------------------------------------------------------------- CPU oracle
-def oracle_sample(seed=4):
-    """A CPU_SAMPLE_ROWS-row slice of the headline workload, prepared for the oracle."""
+def oracle_sample(rows=CPU_SAMPLE_ROWS, seed=4):
+    """A `rows`-row slice of the headline workload, prepared for the oracle."""
     from dynamic_approximate_gemv_b200 import inputs
     from oracle import effort_oracle as O
-    Wn = inputs.weights(CPU_SAMPLE_ROWS, OUT_DIM, seed)
+    Wn = inputs.weights(rows, OUT_DIM, seed)
     prep = O.Prepared(Wn.view(np.uint16), KEEP)
-    vs = [inputs.vector(CPU_SAMPLE_ROWS, 50 + k, "t3") for k in range(4)]
+    vs = [inputs.vector(rows, 50 + k, "t3") for k in range(4)]
     return prep, vs
 
 
-def time_oracle(steps, warmup, min_seconds=0.0):
-    """Oracle matvecs on the row slice; returns us per full matvec (scaled by rows)."""
+def time_oracle(steps, warmup, min_seconds=0.0, rows=CPU_SAMPLE_ROWS):
+    """Oracle matvecs on a `rows`-row slice; returns us per full matvec (time
+    scaled by in_dim / rows), the matvecs done and the seconds they took."""
     from oracle import effort_oracle as O
-    prep, vs = oracle_sample()
+    prep, vs = oracle_sample(rows)
     for k in range(warmup):
         O.effort_gemv(prep, vs[k % len(vs)], EFFORT)
     t0 = time.perf_counter()
@@ -92,26 +93,42 @@ def time_oracle(steps, warmup, min_seconds=0.0):
         O.effort_gemv(prep, vs[done % len(vs)], EFFORT)
         done += 1
     dt = time.perf_counter() - t0
-    scale = IN_DIM / CPU_SAMPLE_ROWS
+    scale = IN_DIM / rows
     return dt / done * scale * 1e6, done, dt
 
 
-def cpu_baseline_record(us, done, dt):
+def cpu_baseline_record(us, done, dt, rows=CPU_SAMPLE_ROWS):
     return {"value": us, "unit": "us", "cores": 1, "kind": "oracle",
-            "sample": f"{done} oracle matvecs on a {CPU_SAMPLE_ROWS}x{OUT_DIM} row slice of the workload "
-                      f"({dt:.1f} s), time scaled by {IN_DIM // CPU_SAMPLE_ROWS} to the full matvec; "
+            "sample": f"{done} oracle matvecs on a {rows}x{OUT_DIM} row slice of the workload "
+                      f"({dt:.1f} s), time scaled by {IN_DIM / rows:g} to the full matvec; "
                       f"numpy, single thread"}
+
+
+REFERENCE_BUDGET_S = 90.0  # the reference arm's timed oracle work, whatever --steps is
+
+
+def reference_rows(steps):
+    """Row-slice size for the reference arm: each of the `steps` timed steps is
+    a bounded sample, so that the whole run takes about REFERENCE_BUDGET_S."""
+    from oracle import effort_oracle as O
+    prep, vs = oracle_sample(32)
+    t0 = time.perf_counter()
+    O.effort_gemv(prep, vs[0], EFFORT)
+    t32 = max(time.perf_counter() - t0, 1e-4)
+    rows = int(32 * REFERENCE_BUDGET_S / (max(steps, 1) * t32))
+    return max(16, min(CPU_SAMPLE_ROWS, rows // 16 * 16))
 
 
 def run_reference(a):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    us, done, dt = time_oracle(a.steps, a.warmup)
+    rows = reference_rows(a.steps)
+    us, done, dt = time_oracle(a.steps, min(a.warmup, 2), rows=rows)
     line = {"metric": METRIC, "value": us, "unit": "us", "n_gpus": a.gpus, "steps": a.steps, "warmup": a.warmup,
             "ms_per_step": us / 1000.0, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
             "dtype": "f64", "data": "synthetic", "impl": "reference", "config": workload_config(),
-            "cpu_baseline": cpu_baseline_record(us, done, dt),
+            "cpu_baseline": cpu_baseline_record(us, done, dt, rows),
             "e2e": {"value": us, "unit": "us", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
