@@ -199,19 +199,49 @@ def rms_norm(y, eps=1e-5):
     return y * torch.rsqrt(torch.mean(y * y) + eps)
 
 
+def effort_for(schedule, layer, name):
+    """Effort of matrix `name` in layer `layer` under `schedule`.
+
+    The pages treat effort as a setting that can change from layer to layer,
+    matrix to matrix and token to token, not only one value for the whole
+    model (the author's replies in Hacker News item 40067677).  A schedule is
+    a number (one effort for every matvec), a mapping keyed by matrix name or
+    by (layer, name), or a callable (layer, name) -> effort.
+    """
+    if callable(schedule):
+        e = schedule(layer, name)
+    elif isinstance(schedule, dict):
+        e = schedule[(layer, name)] if (layer, name) in schedule else schedule[name]
+    else:
+        e = schedule
+    e = float(e)
+    if not 0.0 <= e <= 1.0:
+        raise ValueError(f"effort {e} for layer {layer} matrix {name} is outside [0, 1]")
+    return e
+
+
+# An illustrative per-matrix schedule for the Mistral-7B shapes: the attention
+# projections at 0.5 and the FFN at 0.19, which keeps the parameter-weighted
+# mean effort near 0.25.  The pages give no schedule; this one only exercises
+# the per-matrix setting.
+CHAIN_EQUALIZER = {"q": 0.5, "k": 0.5, "v": 0.5, "o": 0.5, "w1": 0.19, "w3": 0.19, "w2": 0.19}
+
+
 def chain_token(E, mats, x, effort):
     """One token through the stack: per layer x -> q, k, v; q -> o; o -> w1, w3;
-    w1 * w3 -> w2; every matvec input RMS-normalised (no gain)."""
-    for L in mats:
+    w1 * w3 -> w2; every matvec input RMS-normalised (no gain).  `effort` is a
+    schedule (see effort_for)."""
+    for l, L in enumerate(mats):
+        e = {name: effort_for(effort, l, name) for name in L}
         xn = rms_norm(x)
-        q = L["q"].gemv(xn, effort)
-        L["k"].gemv(xn, effort)
-        L["v"].gemv(xn, effort)
-        o = L["o"].gemv(rms_norm(q), effort)
+        q = L["q"].gemv(xn, e["q"])
+        L["k"].gemv(xn, e["k"])
+        L["v"].gemv(xn, e["v"])
+        o = L["o"].gemv(rms_norm(q), e["o"])
         h = rms_norm(o)
-        a = L["w1"].gemv(h, effort)
-        b = L["w3"].gemv(h, effort)
-        x = rms_norm(L["w2"].gemv(rms_norm(a * b), effort))
+        a = L["w1"].gemv(h, e["w1"])
+        b = L["w3"].gemv(h, e["w3"])
+        x = rms_norm(L["w2"].gemv(rms_norm(a * b), e["w2"]))
     return x
 
 
@@ -234,25 +264,32 @@ def measure_chain(E, dev, layers=32, dims=(4096, 1024, 14336), effort=0.25, keep
     x0 = torch.from_numpy(inputs.vector(dims[0], 9)).to(dev)
     s = torch.cuda.Stream(device=dev)
     s.wait_stream(torch.cuda.current_stream(dev))
-    with torch.cuda.stream(s):
-        chain_token(E, mats, x0, effort)
-    torch.cuda.synchronize()
-    gr = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(gr, stream=s):
-        chain_token(E, mats, x0, effort)
-    for _ in range(3):
-        gr.replay()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    reps = 10
-    e0.record()
-    for _ in range(reps):
-        gr.replay()
-    e1.record()
-    torch.cuda.synchronize()
-    us = e0.elapsed_time(e1) * 1000.0 / reps
+
+    def token_us(schedule):
+        with torch.cuda.stream(s):
+            chain_token(E, mats, x0, schedule)
+        torch.cuda.synchronize()
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=s):
+            chain_token(E, mats, x0, schedule)
+        for _ in range(3):
+            gr.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 10
+        e0.record()
+        for _ in range(reps):
+            gr.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        del gr
+        return e0.elapsed_time(e1) * 1000.0 / reps
+
+    us = token_us(effort)
+    us_eq = token_us(CHAIN_EQUALIZER)
+    params = {name: dims[a] * dims[b] for name, a, b in CHAIN_MATS}
+    eq_mean = sum(CHAIN_EQUALIZER[n] * params[n] for n in params) / sum(params.values())
     storage = sum(L[n].info()["device_bytes"] for L in mats for n in L) if hasattr(mats[0]["q"], "info") else None
-    del gr
     for L in mats:
         for n in L:
             L[n].close()
@@ -261,7 +298,9 @@ def measure_chain(E, dev, layers=32, dims=(4096, 1024, 14336), effort=0.25, keep
                         f"effort {effort}; {7 * layers} dependent matvecs per token, RMS-normalised inputs",
             "us_per_token": us, "matvecs_per_token": 7 * layers, "us_per_matvec": us / (7 * layers),
             "dense_roofline_us_per_token_measured_peak": dense_bytes / (hbm_peak()[0] * 1e9) * 1e6,
-            "prepared_bytes": storage}
+            "prepared_bytes": storage,
+            "per_matrix_schedule": {"efforts": CHAIN_EQUALIZER, "parameter_weighted_mean_effort": eq_mean,
+                                    "us_per_token": us_eq}}
 
 
 # ----------------------------------------------------------------- ranks

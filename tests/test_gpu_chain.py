@@ -3,9 +3,11 @@
 The stack follows the Mistral-7B layer pattern at a reduced width: per layer
 q, k, v, o, w1, w3, w2 with every matvec input RMS-normalised, each output
 feeding the next step.  Every matvec of two layers is compared with the oracle
-on the GPU's own input to that step: the cutoff bit for bit, the used count
-exactly, the output within the parity tolerance.  Selection exactness is thus
-defined at every step even though the chain's inputs come from the GPU.
+on the GPU's own input to that step, under one effort for the whole stack and
+under a schedule that changes the effort from matvec to matvec: the cutoff bit
+for bit, the used count exactly, the output within the parity tolerance.
+Selection exactness is thus defined at every step even though the chain's
+inputs come from the GPU.
 """
 import os
 import sys
@@ -54,11 +56,11 @@ def checked_gemv(pm, prep, x, effort):
     return out
 
 
-def test_chain_two_layers_teacher_forced(E):
+def run_chain(E, schedule):
     sys.path.insert(0, ROOT)
     import bench
     dims = (512, 128, 1792)  # d_model, kv width, ffn width (Mistral-7B pattern, scaled by 1/8)
-    layers, effort, keep = 2, 0.25, 0.8
+    layers, keep = 2, 0.8
     mats, preps = [], []
     for l in range(layers):
         L, P = {}, {}
@@ -70,18 +72,35 @@ def test_chain_two_layers_teacher_forced(E):
         preps.append(P)
     try:
         x = torch.from_numpy(inputs.vector(dims[0], 9)).cuda()
-        for L, P in zip(mats, preps):
+        for l, (L, P) in enumerate(zip(mats, preps)):
+            e = {name: bench.effort_for(schedule, l, name) for name in L}
             xn = bench.rms_norm(x)
-            q = checked_gemv(L["q"], P["q"], xn, effort)
-            checked_gemv(L["k"], P["k"], xn, effort)
-            checked_gemv(L["v"], P["v"], xn, effort)
-            o = checked_gemv(L["o"], P["o"], bench.rms_norm(q), effort)
+            q = checked_gemv(L["q"], P["q"], xn, e["q"])
+            checked_gemv(L["k"], P["k"], xn, e["k"])
+            checked_gemv(L["v"], P["v"], xn, e["v"])
+            o = checked_gemv(L["o"], P["o"], bench.rms_norm(q), e["o"])
             h = bench.rms_norm(o)
-            a = checked_gemv(L["w1"], P["w1"], h, effort)
-            b = checked_gemv(L["w3"], P["w3"], h, effort)
-            x = bench.rms_norm(checked_gemv(L["w2"], P["w2"], bench.rms_norm(a * b), effort))
+            a = checked_gemv(L["w1"], P["w1"], h, e["w1"])
+            b = checked_gemv(L["w3"], P["w3"], h, e["w3"])
+            x = bench.rms_norm(checked_gemv(L["w2"], P["w2"], bench.rms_norm(a * b), e["w2"]))
         assert torch.isfinite(x).all()
     finally:
         for L in mats:
             for pm in L.values():
                 pm.close()
+
+
+def test_chain_two_layers_teacher_forced(E):
+    run_chain(E, 0.25)
+
+
+def test_chain_per_matrix_effort_schedule(E):
+    """Effort set matvec by matvec (the pages' per-layer, per-matrix knob):
+    each of the 14 matvecs takes the next effort of a cycle that includes the
+    whole-matrix case, and each is checked against the oracle at its own
+    effort."""
+    sys.path.insert(0, ROOT)
+    import bench
+    cycle = (0.05, 0.15, 0.25, 0.5, 1.0)
+    names = [n for n, _, _ in bench.CHAIN_MATS]
+    run_chain(E, lambda layer, name: cycle[(7 * layer + names.index(name)) % len(cycle)])
