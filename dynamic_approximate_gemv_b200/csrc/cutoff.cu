@@ -46,7 +46,9 @@ struct CutShared {
 
 // Over a complete histogram of B digits (B a multiple of kCutThreads / 32 ...
 // any B up to 4 * kCutThreads): D = max{d : weight of digits >= d reaches
-// krem}, and the weight still needed inside digit D.  Three block barriers.
+// krem}, and the weight still needed inside digit D.  Two block barriers; the
+// caller passes at least one more barrier before cs.sel_* or cs.warp_tot is
+// written again.
 template <int B>
 __device__ void find_crossing(const unsigned* hist, unsigned krem, CutShared& cs, unsigned& digit, unsigned& knew) {
   constexpr int q = (B + kCutThreads - 1) / kCutThreads;  // digits per thread, highest digits first
@@ -89,7 +91,6 @@ __device__ void find_crossing(const unsigned* hist, unsigned krem, CutShared& cs
   __syncthreads();
   digit = cs.sel_digit;
   knew = cs.sel_krem;
-  __syncthreads();
 }
 
 // Cluster-wide radix pass (used when the first-pass bin is crowded).
@@ -124,12 +125,11 @@ __device__ void cluster_radix_pass(cg::cluster_group& cluster, int cl, int crank
   krem = knew;
 }
 
-// Local radix pass over gathered (value, weight) candidates.
+// Local radix pass over gathered (value, weight) candidates.  `hist` (B bins)
+// was zeroed before the last block barrier.
 template <int B>
 __device__ void local_radix_pass(int shift, const unsigned* val, const unsigned short* wt, int n, unsigned* hist,
                                  unsigned& prefix, unsigned& pmask, unsigned& krem, CutShared& cs) {
-  for (int b = threadIdx.x; b < B; b += blockDim.x) hist[b] = 0u;
-  __syncthreads();
   for (int e = threadIdx.x; e < n; e += blockDim.x) {
     const unsigned x = val[e];
     if ((x & pmask) == prefix) atomicAdd(&hist[(x >> shift) & (B - 1)], (unsigned)wt[e]);
@@ -252,24 +252,51 @@ __global__ void __launch_bounds__(kCutThreads, 1) k_cutoff_dispatch(const __grid
     }
     cluster.sync();  // merged slices complete
     {
-      unsigned* full = h0;  // the local histogram is no longer needed: reuse it for the merged copy
-      constexpr int kPerThread = kBins0 / kCutThreads;
-      unsigned x[kPerThread];
+      // The crossing of the merged histogram, read straight from the owners'
+      // slices: thread j owns digits [kBins0 - 4 (j + 1), kBins0 - 4 j) (thread
+      // 0 the highest), four adjacent bins of one slice fetched with one
+      // 16-byte remote load and scanned in registers.
+      static_assert(kBins0 == 4 * kCutThreads, "four first-digit bins per thread");
+      const int ln = threadIdx.x & 31, wp = threadIdx.x >> 5;
+      const int hi = kBins0 - 4 * (int)threadIdx.x, b0 = hi - 4;
+      const uint4 q = *reinterpret_cast<const uint4*>(cluster.map_shared_rank(own, b0 / per) + (b0 % per));
+      const unsigned local = q.x + q.y + q.z + q.w;
+      unsigned x = local;  // inclusive scan over threads in order (= descending digits)
 #pragma unroll
-      for (int u = 0; u < kPerThread; ++u) {
-        const int b = threadIdx.x + u * kCutThreads;
-        x[u] = *(cluster.map_shared_rank(own, b / per) + (b % per));
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+        if (ln >= o) x += y;
+      }
+      if (ln == 31) cs.warp_tot[wp] = x;
+      __syncthreads();
+      unsigned wt = cs.warp_tot[ln];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned y = __shfl_up_sync(0xFFFFFFFFu, wt, o);
+        if (ln >= o) wt += y;
+      }
+      const unsigned before = __shfl_sync(0xFFFFFFFFu, wt, wp > 0 ? wp - 1 : 0) * (wp > 0 ? 1u : 0u);
+      unsigned cum = before + x - local;  // weight of all digits above this thread's
+      if (cum < Kt && cum + local >= Kt) {
+        const unsigned hv[4] = {q.w, q.z, q.y, q.x};  // digits hi - 1 ... hi - 4
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          if (cum + hv[u] >= Kt) {
+            cs.sel_digit = (unsigned)(hi - 1 - u);
+            cs.sel_krem = Kt - cum;
+            break;
+          }
+          cum += hv[u];
+        }
       }
       __syncthreads();
-#pragma unroll
-      for (int u = 0; u < kPerThread; ++u) full[threadIdx.x + u * kCutThreads] = x[u];
-      __syncthreads();
     }
-    unsigned digit, knew;
-    find_crossing<kBins0>(h0, Kt, cs, digit, knew);
-    prefix = digit << 19;
+    prefix = cs.sel_digit << 19;
     pmask = (unsigned)(kBins0 - 1) << 19;
-    krem = knew;
+    krem = cs.sel_krem;
+    // the local passes' histograms (h0 is free since the merge barrier)
+    static_assert(kBins1 + kBins2 <= kBins0, "local-pass histograms fit the first-pass one");
+    for (int b = threadIdx.x; b < kBins1 + kBins2; b += blockDim.x) h0[b] = 0u;
     // ---- this CTA's entries in the chosen bin (one atomic per warp)
     for (int e = threadIdx.x; e < ne; e += blockDim.x) {
       const int k = __float2int_rd(((float)e + 0.5f) * rcp_rp);
@@ -339,7 +366,7 @@ __global__ void __launch_bounds__(kCutThreads, 1) k_cutoff_dispatch(const __grid
       split_exit = true;
       __syncthreads();
       local_radix_pass<kBins1>(9, gval, gwt, (int)total, h0, prefix, pmask, krem, cs);
-      local_radix_pass<kBins2>(0, gval, gwt, (int)total, h0, prefix, pmask, krem, cs);
+      local_radix_pass<kBins2>(0, gval, gwt, (int)total, h0 + kBins1, prefix, pmask, krem, cs);
     } else {
       cluster_radix_pass<kBins1>(cluster, cl, crank, 9, chart, RP, nr, s_pw, h1, m1, prefix, pmask, krem, cs);
       cluster_radix_pass<kBins2>(cluster, cl, crank, 0, chart, RP, nr, s_pw, h2, m2, prefix, pmask, krem, cs);
