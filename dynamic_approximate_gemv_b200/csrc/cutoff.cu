@@ -192,6 +192,14 @@ __global__ void __launch_bounds__(kCutThreads, 1) k_cutoff_dispatch(const __grid
 
   int mode = jb.mode;
   if (threadIdx.x == 0) cs.ncand = 0u;
+  // the first-pass histogram and this CTA's merged slice, zeroed while the
+  // chart's loads are in flight (the barrier after the chart covers both)
+  const int per = kBins0 / cl;
+  unsigned* own = mg0;  // this CTA's merged slice lives at the start of the shared area
+  if (mode == kModeSelect) {
+    for (int b = threadIdx.x; b < kBins0; b += blockDim.x) h0[b] = 0u;
+    for (int b = threadIdx.x; b < per; b += blockDim.x) own[b] = 0u;
+  }
   // ---- v and probes (one thread per row), and an L2 prefetch of the row's
   // checkpoint magnitudes for the dispatch
   bool bad = false;
@@ -228,13 +236,8 @@ __global__ void __launch_bounds__(kCutThreads, 1) k_cutoff_dispatch(const __grid
   if (mode == kModeSelect) {
     // ---- first digit, cluster-wide.  Local weighted histogram; its nonzero
     // bins are added into the owner CTA's slice (bin / (kBins0 / cl)) with
-    // distributed shared memory atomics; after one cluster barrier every CTA
-    // reads the whole merged histogram.
-    const int per = kBins0 / cl;
-    unsigned* own = mg0;  // this CTA's merged slice lives at the start of the shared area
-    for (int b = threadIdx.x; b < kBins0; b += blockDim.x) h0[b] = 0u;
-    for (int b = threadIdx.x; b < per; b += blockDim.x) own[b] = 0u;
-    __syncthreads();
+    // distributed shared memory atomics; after one cluster barrier each thread
+    // reads its four bins of the merged histogram from their owner's slice.
     // chart entry e = k * RP + r (column-major); k from a float reciprocal,
     // exact for e < 2^16 and RP <= 2^12
     const int ne = kP * RP;
@@ -403,7 +406,7 @@ __global__ void __launch_bounds__(kCutThreads, 1) k_cutoff_dispatch(const __grid
         // none); fl32(|v_i| * m) is non-decreasing in m, so |w| >= tau <=> used.
         // Start from the fp16 rounding of c / |v_i| and settle it with exact
         // product tests; a bisection over all magnitudes covers the rest.
-        const float q = c * (1.0f / av);  // inf when av == 0
+        const float q = __fdividef(c, av);  // a guess only (inf when av == 0; c > 0 here)
         unsigned lo = 0u, hi = 0x7C00u;
         if (q < 65504.0f) {
           const unsigned g = (unsigned)__half_as_ushort(__float2half_rd(q)) & 0x7FFFu;
@@ -424,6 +427,7 @@ __global__ void __launch_bounds__(kCutThreads, 1) k_cutoff_dispatch(const __grid
         tau = lo;
         // probes narrow the rank range of the row's boundary
         int last_sel = -1, first_unsel = n;
+#pragma unroll
         for (int k = 0; k < kP; ++k) {
           const int rk = s_prank[k];
           if (rk < 0) continue;
