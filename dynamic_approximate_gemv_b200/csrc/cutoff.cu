@@ -40,6 +40,7 @@ struct CutShared {
   unsigned sel_digit;
   unsigned sel_krem;
   unsigned ncand;       // this CTA's entries in the first-pass bin
+  unsigned ncnt[16];    // every cluster CTA's ncand, stored here by that CTA
   unsigned cand_off[17];
   unsigned cand_total;
 };
@@ -199,6 +200,9 @@ __global__ void __launch_bounds__(kCutThreads, 1) k_cutoff_dispatch(const __grid
   if (mode == kModeSelect) {
     for (int b = threadIdx.x; b < kBins0; b += blockDim.x) h0[b] = 0u;
     for (int b = threadIdx.x; b < per; b += blockDim.x) own[b] = 0u;
+    // split cluster barrier: arrive now (this CTA's slice is zeroed), wait
+    // just before the first remote atomic into another CTA's slice
+    asm volatile("barrier.cluster.arrive.release.aligned;\n" ::: "memory");
   }
   // ---- v and probes (one thread per row), and an L2 prefetch of the row's
   // checkpoint magnitudes for the dispatch
@@ -248,7 +252,8 @@ __global__ void __launch_bounds__(kCutThreads, 1) k_cutoff_dispatch(const __grid
       const int wk = s_pw[k];
       if (r < nr && wk > 0) atomicAdd(&h0[(chart[e] >> 19) & (kBins0 - 1)], (unsigned)wk);
     }
-    cluster.sync();  // every CTA's slice is zeroed and its local histogram complete
+    __syncthreads();  // the local histogram is complete
+    asm volatile("barrier.cluster.wait.acquire.aligned;\n" ::: "memory");  // every CTA's slice is zeroed
     for (int b = threadIdx.x; b < kBins0; b += blockDim.x) {
       const unsigned x = h0[b];
       if (x) atomicAdd(cluster.map_shared_rank(own, b / per) + (b % per), x);
@@ -321,10 +326,13 @@ __global__ void __launch_bounds__(kCutThreads, 1) k_cutoff_dispatch(const __grid
       }
     }
     __syncthreads();
+    // this CTA's list length into every CTA's table (the barrier below
+    // publishes it), so that no CTA reads the lengths remotely afterwards
+    if ((int)threadIdx.x < cl) *cluster.map_shared_rank(&cs.ncnt[crank], (int)threadIdx.x) = cs.ncand;
     cluster.sync();  // every list complete; no CTA reads another's merged slice any more
-    if (threadIdx.x < 32) {  // the cl list lengths, read in parallel, and their offsets
+    if (threadIdx.x < 32) {  // the cl list lengths and their offsets
       const int ln = threadIdx.x;
-      const unsigned nc = (ln < cl) ? *cluster.map_shared_rank(&cs.ncand, ln) : 0u;
+      const unsigned nc = (ln < cl) ? cs.ncnt[ln] : 0u;
       const bool over = __any_sync(0xFFFFFFFFu, nc > (unsigned)kCandLocal);
       unsigned incl = nc;
 #pragma unroll
