@@ -204,31 +204,43 @@ __global__ void __launch_bounds__(kCutThreads, 1) k_cutoff_dispatch(const __grid
     // just before the first remote atomic into another CTA's slice
     asm volatile("barrier.cluster.arrive.release.aligned;\n" ::: "memory");
   }
-  // ---- v and probes (one thread per row), and an L2 prefetch of the row's
-  // checkpoint magnitudes for the dispatch
-  bool bad = false;
+  // ---- before the preceding grid of the stream has completed: only the
+  // prepared matrix (never written by a call) and shared memory are touched.
+  // The probes go into the chart area as floats; the rows' checkpoint
+  // magnitudes are prefetched into L2 for the dispatch.
   for (int r = threadIdx.x; r < nr; r += blockDim.x) {
     const int i = i0 + r;
-    uint4 p0 = make_uint4(0, 0, 0, 0), p1 = p0;
     if (mode == kModeSelect) {
-      p0 = reinterpret_cast<const uint4*>(probes + (size_t)i * kP)[0];
-      p1 = reinterpret_cast<const uint4*>(probes + (size_t)i * kP)[1];
-    }
-    const float x = (vdtype == 1) ? __half2float(reinterpret_cast<const __half*>(vptr)[i])
-                                  : reinterpret_cast<const float*>(vptr)[i];
-    const char* ck = reinterpret_cast<const char*>(ckmag + (size_t)i * (C + 1));
-    for (int b = 0; b < (C + 1) * 2; b += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(ck + b));
-    if (!isfinite(x)) bad = true;
-    vs[r] = x;
-    if (mode == kModeSelect) {
-      const float av = fabsf(x);
+      const uint4 p0 = reinterpret_cast<const uint4*>(probes + (size_t)i * kP)[0];
+      const uint4 p1 = reinterpret_cast<const uint4*>(probes + (size_t)i * kP)[1];
       const unsigned short* ph0 = reinterpret_cast<const unsigned short*>(&p0);
       const unsigned short* ph1 = reinterpret_cast<const unsigned short*>(&p1);
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
-        chart[(size_t)k * RP + r] = __float_as_uint(__fmul_rn(av, __half2float(__ushort_as_half(ph0[k]))));
-        chart[(size_t)(8 + k) * RP + r] = __float_as_uint(__fmul_rn(av, __half2float(__ushort_as_half(ph1[k]))));
+        chart[(size_t)k * RP + r] = __float_as_uint(__half2float(__ushort_as_half(ph0[k])));
+        chart[(size_t)(8 + k) * RP + r] = __float_as_uint(__half2float(__ushort_as_half(ph1[k])));
       }
+    }
+    const char* ck = reinterpret_cast<const char*>(ckmag + (size_t)i * (C + 1));
+    for (int b = 0; b < (C + 1) * 2; b += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(ck + b));
+  }
+  // the preceding grid may produce v and may still read this call's scratch:
+  // everything below comes after its completion
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  // ---- v, and the chart x_ik = fl32(|v_i| * p_ik) (each thread rescales the
+  // probes of its own rows in place)
+  bool bad = false;
+  for (int r = threadIdx.x; r < nr; r += blockDim.x) {
+    const int i = i0 + r;
+    const float x = (vdtype == 1) ? __half2float(reinterpret_cast<const __half*>(vptr)[i])
+                                  : reinterpret_cast<const float*>(vptr)[i];
+    if (!isfinite(x)) bad = true;
+    vs[r] = x;
+    if (mode == kModeSelect) {
+      const float av = fabsf(x);
+#pragma unroll
+      for (int k = 0; k < kP; ++k)
+        chart[(size_t)k * RP + r] = __float_as_uint(__fmul_rn(av, __uint_as_float(chart[(size_t)k * RP + r])));
     }
   }
   if (bad) atomicOr(status, kStatusNonfiniteV);
@@ -569,13 +581,18 @@ cudaError_t launch_cutoff_t(const Jobs<NJ>& jobs, int njobs, int I, int cl, cuda
   cfg.blockDim = dim3(kCutThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = (unsigned)cl;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  // may start once the preceding grid allows it (the multiply of an earlier
+  // call does so as soon as all its CTAs run); the kernel waits for that
+  // grid's completion before it reads v or touches the scratch
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, k_cutoff_dispatch<NJ>, jobs, cl);
 }
 
