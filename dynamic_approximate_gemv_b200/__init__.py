@@ -55,6 +55,7 @@ def lib():
             "effort_gemv": [vp, vp, f32, vp, vp],
             "effort_gemv_ex": [vp, vp, ctypes.c_int, f32, vp, vp, vp, vp, vp],
             "effort_gemv_split": [vp, vp, ctypes.c_int, f32, vp, vp, vp, vp, vp],
+            "effort_gemv_host": [vp, vp, ctypes.c_int, f32, vp, vp],
             "effort_gemv_static": [vp, vp, ctypes.c_int, f32, vp, vp, vp, vp, vp],
             "effort_check": [vp],
             "effort_workspace_create": [i64, i64, i32, ctypes.POINTER(vp)],
@@ -144,6 +145,26 @@ class PreparedMatrix:
                     raise ValueError(f"{nm} must be {dt} of shape {shp}")
         _check(lib().effort_gemv_ex(self._h, _ptr(v), _vdtype(v), ctypes.c_float(effort), _ptr(out), _ptr(cutoff),
                                     _ptr(count), _ptr(rowlen), _stream(v.device)), "effort_gemv")
+        return out
+
+    def gemv_host(self, v, effort, out=None):
+        """gemv on host tensors: v (float32 or float16 [in_dim]) is copied to the
+        device, the matvec runs, and out (float32 [out_dim], host) is copied
+        back, all on the current stream of the handle's device.  Pinned
+        (page-locked) tensors keep the copies asynchronous.  out is valid once
+        that stream has passed the call (e.g. torch.cuda.synchronize())."""
+        if not (isinstance(v, torch.Tensor) and v.device.type == "cpu" and v.is_contiguous()):
+            raise ValueError("v must be a contiguous host tensor")
+        if v.shape != (self.in_dim,):
+            raise ValueError("v has the wrong shape")
+        if out is None:
+            out = torch.empty(self.out_dim, dtype=torch.float32, pin_memory=True)
+        if not (isinstance(out, torch.Tensor) and out.device.type == "cpu" and out.is_contiguous()):
+            raise ValueError("out must be a contiguous host tensor")
+        if out.dtype != torch.float32 or out.shape != (self.out_dim,):
+            raise ValueError("out must be float32 [out_dim]")
+        _check(lib().effort_gemv_host(self._h, _ptr(v), _vdtype(v), ctypes.c_float(effort), _ptr(out),
+                                      _stream(self.device)), "effort_gemv_host")
         return out
 
     def gemv_static(self, v, effort, out=None, cutoff=None, count=None, status=None):

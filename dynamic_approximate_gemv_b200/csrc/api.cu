@@ -166,6 +166,9 @@ struct DeviceGuard {
 
 }  // namespace
 
+// Offset of out inside effort_gemv_host's staging buffer (v first).
+static size_t stage_out_offset(int I) { return ((size_t)I * 4 + 255) / 256 * 256; }
+
 struct effort_handle_s {
   int dev = 0;
   Geometry g = {};
@@ -176,6 +179,7 @@ struct effort_handle_s {
   size_t storage_bytes = 0;
   WsBlock ws;
   WsPtrs slot = {};
+  void* stage = nullptr;  // device staging of effort_gemv_host: v (in_dim x 4 B), then out (out_dim x 4 B)
   cudaStream_t last_stream = nullptr;
 };
 
@@ -305,6 +309,13 @@ effort_status_t effort_prepare(const void* W, int64_t in_dim, int64_t out_dim, f
     delete h;
     return st;
   }
+  if (cudaMalloc(&h->stage, stage_out_offset(g.I) + (size_t)g.O * 4) != cudaSuccess) {
+    cudaGetLastError();
+    cudaFree(h->ws.base);
+    cudaFree(h->storage);
+    delete h;
+    return EFFORT_ERR_NOMEM;
+  }
   *out_handle = h;
   return EFFORT_OK;
 }
@@ -371,6 +382,29 @@ effort_status_t effort_gemv_split(effort_handle_t h, const void* v, effort_dtype
   }
   if (e == cudaSuccess) e = launch_mac(jobs, h->g.T, h->g.S, s);
   if (e != cudaSuccess) {
+    cudaGetLastError();
+    return EFFORT_ERR_CUDA;
+  }
+  return EFFORT_OK;
+}
+
+effort_status_t effort_gemv_host(effort_handle_t h, const void* v_host, effort_dtype_t v_dtype, float effort,
+                                 float* out_host, void* stream) {
+  if (!h || !v_host || !out_host) return EFFORT_ERR_ARG;
+  if (v_dtype != EFFORT_F32 && v_dtype != EFFORT_F16) return EFFORT_ERR_ARG;
+  if (!effort_ok(effort)) return EFFORT_ERR_ARG;
+  DeviceGuard guard(h->dev);
+  cudaStream_t s = (cudaStream_t)stream;
+  void* d_v = h->stage;
+  float* d_out = reinterpret_cast<float*>(static_cast<char*>(h->stage) + stage_out_offset(h->g.I));
+  const size_t vbytes = (size_t)h->g.I * (v_dtype == EFFORT_F16 ? 2 : 4);
+  if (cudaMemcpyAsync(d_v, v_host, vbytes, cudaMemcpyHostToDevice, s) != cudaSuccess) {
+    cudaGetLastError();
+    return EFFORT_ERR_CUDA;
+  }
+  const effort_status_t st = effort_gemv_ex(h, d_v, v_dtype, effort, d_out, nullptr, nullptr, nullptr, stream);
+  if (st != EFFORT_OK) return st;
+  if (cudaMemcpyAsync(out_host, d_out, (size_t)h->g.O * 4, cudaMemcpyDeviceToHost, s) != cudaSuccess) {
     cudaGetLastError();
     return EFFORT_ERR_CUDA;
   }
@@ -527,6 +561,7 @@ effort_status_t effort_destroy(effort_handle_t h) {
   {
     DeviceGuard guard(h->dev);
     cudaStreamSynchronize(h->last_stream);
+    cudaFree(h->stage);
     cudaFree(h->ws.base);
     cudaFree(h->storage);
   }

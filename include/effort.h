@@ -104,6 +104,26 @@ effort_status_t effort_gemv_ex(effort_handle_t h, const void* v, effort_dtype_t 
                                void* stream);
 
 /*
+ * effort_gemv_host -- effort_gemv_ex on HOST buffers, for callers that hold v
+ *   and want out in host memory.  The pages have no counterpart: this is a
+ *   library service around the same matvec.  On `stream`, in order: one
+ *   cudaMemcpyAsync of v (in_dim elements of v_dtype) into the handle's
+ *   device staging buffer, the same two kernels as effort_gemv_ex, and one
+ *   cudaMemcpyAsync of out (out_dim fp32) back to out_host.
+ *   v_host, out_host: host memory, non-NULL.  Page-locked memory
+ *     (cudaHostAlloc, cudaHostRegister) keeps the copies asynchronous; with
+ *     pageable memory CUDA stages the copies and they may block the host.
+ *   The call does not synchronise: out_host holds the result once the stream
+ *   has passed this call (cudaStreamSynchronize, an event).  The caller must
+ *   not modify v_host or read out_host before then.
+ *   The staging buffer (in_dim x 4 + out_dim x 4 bytes) is allocated by
+ *   effort_prepare and belongs to the handle: calls on one handle must be
+ *   ordered (one stream), like the handle's workspace.
+ */
+effort_status_t effort_gemv_host(effort_handle_t h, const void* v_host, effort_dtype_t v_dtype, float effort,
+                                 float* out_host, void* stream);
+
+/*
  * effort_gemv_split -- effort_gemv_ex that also records `mid_event` (a
  *   cudaEvent_t passed as void*, created by the caller) on the stream between
  *   the cutoff/dispatch kernel and the multiply kernel, so that each phase can

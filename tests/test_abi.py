@@ -26,7 +26,8 @@ def declared_functions():
 
 def test_header_declares_the_boundary():
     names = declared_functions()
-    for must in ("effort_prepare", "effort_gemv", "effort_gemv_ex", "effort_gemv_batched", "effort_destroy",
+    for must in ("effort_prepare", "effort_gemv", "effort_gemv_ex", "effort_gemv_host", "effort_gemv_batched",
+                 "effort_destroy",
                  "effort_dense_gemv", "effort_workspace_create", "effort_status_string"):
         assert must in names
 
@@ -57,6 +58,7 @@ def test_argument_errors_need_no_device(L):
     assert L.effort_prepare(fake, 4, 10, ctypes.c_float(0.04), None, ctypes.byref(h)) == 1  # keeps nothing
     assert L.effort_gemv(None, fake, ctypes.c_float(0.5), fake, None) == 1
     assert L.effort_gemv_ex(None, fake, 0, ctypes.c_float(0.5), fake, None, None, None, None) == 1
+    assert L.effort_gemv_host(None, fake, 0, ctypes.c_float(0.5), fake, None) == 1
     assert L.effort_check(None) == 1
     assert L.effort_destroy(None) == 1
     w = vp()

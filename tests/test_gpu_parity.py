@@ -166,6 +166,26 @@ def test_fp16_vector(E):
     check_call(E, prep, pm, v, 0.25)
 
 
+@pytest.mark.parametrize("dtype", [np.float32, np.float16])
+def test_host_buffers_match_device_call(E, dtype):
+    """effort_gemv_host (host v in, host out back) gives the device call's
+    output bit for bit, and so the oracle's within the contract."""
+    _, prep, pm = make(E, 1000, 1300, 21, keep=0.9)
+    v_np = inputs.vector(1000, 22, "t3", dtype=dtype)
+    v_host = torch.from_numpy(v_np).pin_memory()
+    out_host = torch.full((1300,), float("nan"), dtype=torch.float32).pin_memory()
+    pm.gemv_host(v_host, 0.3, out_host)
+    torch.cuda.synchronize()
+    dev_out = pm.gemv(torch.from_numpy(v_np).cuda(), 0.3).cpu()
+    assert torch.equal(out_host, dev_out)
+    assert_out_close(out_host.numpy(), O.effort_gemv(prep, v_np, 0.3).out)
+    # pageable host memory works too (the copies are staged by CUDA)
+    out2 = torch.zeros(1300, dtype=torch.float32)
+    pm.gemv_host(torch.from_numpy(v_np), 0.3, out2)
+    torch.cuda.synchronize()
+    assert torch.equal(out2, dev_out)
+
+
 def test_one_hot_rows_product_by_product(E):
     Wn, prep, pm = make(E, 64, 700, 13)
     for i in (0, 17, 63):
