@@ -10,8 +10,9 @@
 //   topK    c = max{x : sum of probe weights of chart entries >= x is >= K}.
 //           Weighted radix select over the bit patterns.  The first digit
 //           (bits 30..19) is chosen cluster-wide: CTA-local weighted
-//           histograms are summed by every CTA through distributed shared
-//           memory.  Each CTA then lists its chart entries that fall in the
+//           histograms are summed into per-CTA slices through distributed
+//           shared memory, and every CTA reads the slices to find the
+//           crossing bin.  Each CTA then lists its chart entries that fall in the
 //           chosen bin, every CTA gathers all lists and finishes the select
 //           locally (bits 18..9, then 8..0); all CTAs reach the same c.  If the
 //           bin holds too many entries, the last two digits are also chosen
@@ -27,6 +28,11 @@
 //           buckets), rows whose largest product is below c are off.  Records
 //           {v_i, tau_i, row} of a 32-row group are written sparse rows first,
 //           then dense rows.
+//
+// Launch: programmatic, behind the preceding grid of the stream.  Before
+// waiting on that grid the kernel touches only the prepared matrix (probes,
+// checkpoint rows) and its shared memory; v, which that grid may produce, and
+// the scratch, which an earlier call's multiply may still read, come after.
 #include <cooperative_groups.h>
 
 #include "effort_internal.cuh"
