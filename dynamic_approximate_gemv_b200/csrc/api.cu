@@ -166,6 +166,18 @@ struct DeviceGuard {
 
 }  // namespace
 
+// Device address of page-locked host memory mapped into the device's address
+// space (cudaHostAlloc, cudaMallocHost, cudaHostRegister with mapping), else
+// nullptr (pageable memory, device memory, unknown pointers).
+static void* mapped_host_pointer(const void* p) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  return (a.type == cudaMemoryTypeHost) ? a.devicePointer : nullptr;
+}
+
 // Offset of out inside effort_gemv_host's staging buffer (v first).
 static size_t stage_out_offset(int I) { return ((size_t)I * 4 + 255) / 256 * 256; }
 
@@ -395,16 +407,22 @@ effort_status_t effort_gemv_host(effort_handle_t h, const void* v_host, effort_d
   if (!effort_ok(effort)) return EFFORT_ERR_ARG;
   DeviceGuard guard(h->dev);
   cudaStream_t s = (cudaStream_t)stream;
-  void* d_v = h->stage;
-  float* d_out = reinterpret_cast<float*>(static_cast<char*>(h->stage) + stage_out_offset(h->g.I));
+  // page-locked memory mapped into the device's address space is read and
+  // written in place by the kernels; other host memory goes through the
+  // staging buffer with one copy each way
+  void* mv = mapped_host_pointer(v_host);
+  void* mo = mapped_host_pointer(out_host);
+  void* d_v = mv ? mv : h->stage;
+  float* d_out = mo ? static_cast<float*>(mo)
+                    : reinterpret_cast<float*>(static_cast<char*>(h->stage) + stage_out_offset(h->g.I));
   const size_t vbytes = (size_t)h->g.I * (v_dtype == EFFORT_F16 ? 2 : 4);
-  if (cudaMemcpyAsync(d_v, v_host, vbytes, cudaMemcpyHostToDevice, s) != cudaSuccess) {
+  if (!mv && cudaMemcpyAsync(d_v, v_host, vbytes, cudaMemcpyHostToDevice, s) != cudaSuccess) {
     cudaGetLastError();
     return EFFORT_ERR_CUDA;
   }
   const effort_status_t st = effort_gemv_ex(h, d_v, v_dtype, effort, d_out, nullptr, nullptr, nullptr, stream);
   if (st != EFFORT_OK) return st;
-  if (cudaMemcpyAsync(out_host, d_out, (size_t)h->g.O * 4, cudaMemcpyDeviceToHost, s) != cudaSuccess) {
+  if (!mo && cudaMemcpyAsync(out_host, d_out, (size_t)h->g.O * 4, cudaMemcpyDeviceToHost, s) != cudaSuccess) {
     cudaGetLastError();
     return EFFORT_ERR_CUDA;
   }

@@ -106,13 +106,17 @@ effort_status_t effort_gemv_ex(effort_handle_t h, const void* v, effort_dtype_t 
 /*
  * effort_gemv_host -- effort_gemv_ex on HOST buffers, for callers that hold v
  *   and want out in host memory.  The pages have no counterpart: this is a
- *   library service around the same matvec.  On `stream`, in order: one
- *   cudaMemcpyAsync of v (in_dim elements of v_dtype) into the handle's
- *   device staging buffer, the same two kernels as effort_gemv_ex, and one
- *   cudaMemcpyAsync of out (out_dim fp32) back to out_host.
- *   v_host, out_host: host memory, non-NULL.  Page-locked memory
- *     (cudaHostAlloc, cudaHostRegister) keeps the copies asynchronous; with
- *     pageable memory CUDA stages the copies and they may block the host.
+ *   library service around the same matvec.  On `stream`, in order, the same
+ *   two kernels as effort_gemv_ex, with v (in_dim elements of v_dtype) and
+ *   out (out_dim fp32) moved across the host link as follows:
+ *   - page-locked memory mapped into the device's address space (cudaHostAlloc,
+ *     cudaMallocHost, cudaHostRegister with mapping; cudaPointerGetAttributes
+ *     decides) is read (v) and written (out) in place by the kernels, with no
+ *     copy operation;
+ *   - other host memory goes through the handle's device staging buffer, with
+ *     one cudaMemcpyAsync before the kernels (v) and one after (out); CUDA
+ *     stages pageable copies, which may block the host.
+ *   v_host, out_host: host memory, non-NULL.
  *   The call does not synchronise: out_host holds the result once the stream
  *   has passed this call (cudaStreamSynchronize, an event).  The caller must
  *   not modify v_host or read out_host before then.

@@ -169,7 +169,8 @@ def test_fp16_vector(E):
 @pytest.mark.parametrize("dtype", [np.float32, np.float16])
 def test_host_buffers_match_device_call(E, dtype):
     """effort_gemv_host (host v in, host out back) gives the device call's
-    output bit for bit, and so the oracle's within the contract."""
+    output bit for bit, and so the oracle's within the contract, both for
+    pinned buffers (accessed in place) and pageable ones (copied)."""
     _, prep, pm = make(E, 1000, 1300, 21, keep=0.9)
     v_np = inputs.vector(1000, 22, "t3", dtype=dtype)
     v_host = torch.from_numpy(v_np).pin_memory()
@@ -179,11 +180,19 @@ def test_host_buffers_match_device_call(E, dtype):
     dev_out = pm.gemv(torch.from_numpy(v_np).cuda(), 0.3).cpu()
     assert torch.equal(out_host, dev_out)
     assert_out_close(out_host.numpy(), O.effort_gemv(prep, v_np, 0.3).out)
-    # pageable host memory works too (the copies are staged by CUDA)
+    # pageable host memory goes through the staging buffer and copies
     out2 = torch.zeros(1300, dtype=torch.float32)
     pm.gemv_host(torch.from_numpy(v_np), 0.3, out2)
     torch.cuda.synchronize()
     assert torch.equal(out2, dev_out)
+    # pinned buffers are read and written in place: new contents of the same
+    # buffers between calls are seen, call after call
+    for seed in (23, 24, 25):
+        w_np = inputs.vector(1000, seed, "normal", dtype=dtype)
+        v_host.copy_(torch.from_numpy(w_np))
+        pm.gemv_host(v_host, 0.3, out_host)
+        torch.cuda.synchronize()
+        assert torch.equal(out_host, pm.gemv(torch.from_numpy(w_np).cuda(), 0.3).cpu())
 
 
 def test_one_hot_rows_product_by_product(E):
