@@ -22,6 +22,7 @@ cudaError_t launch_mac_batch(const Jobs<kMaxJobs>& jobs, int njobs, int T, int S
 cudaError_t launch_dense(const uint16_t* W, int I, int O, const void* v, int vdtype, float* out, float* part,
                          unsigned* tilecnt, int T, int S, cudaStream_t stream);
 int mac_ctas_per_sm();
+int dense_ctas_per_sm();
 cudaError_t init_kernel_attributes();
 size_t cutoff_max_dynamic_smem();
 int cutoff_max_clusters(int cl, size_t smem);
@@ -94,7 +95,8 @@ effort_status_t make_geometry(int64_t I, int64_t O, Geometry* g) {
     if (f > 0.0 && f <= 1.0) frac = f;
   }
   g->dense_q16 = (int)(frac * 65536.0 + 0.5);
-  int Sd = (g_num_sms * 8) / g->T;
+  // the dense baseline's T x Sd CTAs fill the SMs once as well
+  int Sd = (g_num_sms * dense_ctas_per_sm()) / g->T;
   if (Sd < 1) Sd = 1;
   if (Sd > (int)((I + 7) / 8)) Sd = (int)((I + 7) / 8);
   if (Sd < 1) Sd = 1;

@@ -77,6 +77,17 @@ __global__ void __launch_bounds__(kDenseThreads) k_dense_gemv(const uint16_t* __
   }
 }
 
+// Resident CTAs of the dense baseline per SM (its registers allow fewer than
+// its thread count would).
+int dense_ctas_per_sm() {
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_dense_gemv<float>, kDenseThreads, 0) != cudaSuccess) {
+    cudaGetLastError();
+    return 1;
+  }
+  return n > 0 ? n : 1;
+}
+
 cudaError_t launch_dense(const uint16_t* W, int I, int O, const void* v, int vdtype, float* out, float* part,
                          unsigned* tilecnt, int T, int S, cudaStream_t stream) {
   const dim3 grid((unsigned)(T * S));
