@@ -11,7 +11,7 @@
 namespace effort {
 
 template <typename VT>
-__global__ void __launch_bounds__(kDenseThreads) k_dense_gemv(const uint16_t* __restrict__ W, int I, int O,
+__global__ void __launch_bounds__(kDenseThreads, 4) k_dense_gemv(const uint16_t* __restrict__ W, int I, int O,
                                                               const VT* __restrict__ v, float* out, float* part,
                                                               unsigned* tilecnt, int T, int S) {
   constexpr int kW = kDenseThreads / 32;
