@@ -215,6 +215,28 @@ def test_repeat_calls_are_deterministic(E):
         assert torch.equal(pm.gemv(v, 0.25), first)
 
 
+def test_back_to_back_calls_on_one_handle(E):
+    """Calls queued back to back on one handle and stream, with no host sync:
+    each call's cutoff starts during the previous call's multiply and reuses
+    its scratch.  Every output must equal the same call made alone."""
+    _, prep, pm = make(E, 2048, 3072, 31)
+    vs = [torch.from_numpy(inputs.vector(2048, 40 + k, "t3" if k % 2 else "normal")).cuda() for k in range(4)]
+    efforts = [0.25, 0.1, 0.5, 0.25, 1.0, 0.05, 0.3, 0.25]
+    alone = []
+    for k, e in enumerate(efforts):
+        alone.append(pm.gemv(vs[k % 4], e).clone())
+        torch.cuda.synchronize()
+    outs = [torch.empty(3072, device="cuda") for _ in efforts]
+    for rep in range(3):
+        for k, e in enumerate(efforts):
+            pm.gemv(vs[k % 4], e, out=outs[k])
+        torch.cuda.synchronize()
+        for k in range(len(efforts)):
+            assert torch.equal(outs[k], alone[k]), (rep, k)
+    ref = O.effort_gemv(prep, vs[1].cpu().numpy(), efforts[1])
+    assert_out_close(alone[1].cpu().numpy(), ref.out)
+
+
 def test_effort_sweep_4096_square(E):
     _, prep, pm = make(E, 4096, 4096, 2)
     v = inputs.vector(4096, 3, dtype=np.float16)
