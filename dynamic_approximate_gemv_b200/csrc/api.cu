@@ -86,10 +86,12 @@ effort_status_t make_geometry(int64_t I, int64_t O, Geometry* g) {
   if (S > g->G) S = g->G;
   g->S = S;
   // rows whose surely-used share reaches this fraction are read from the dense
-  // copy (2 B per weight, register accumulation) instead of their buckets; a
-  // dense tile row costs about as many instructions as a quarter of it read
-  // through the buckets, which puts the break-even near 0.3
-  double frac = 0.3;
+  // copy (2 B per weight, register accumulation) instead of their buckets.  A
+  // sparse row-tile's short prefix rounds up to whole sectors twice (values,
+  // columns), so a row read through its buckets costs more per used product
+  // than its byte count suggests; measured step times are flat from 0.1 to
+  // 0.2 and rise above that
+  double frac = 0.2;
   if (const char* env = getenv("EFFORT_DENSE_FRACTION")) {
     const double f = atof(env);
     if (f > 0.0 && f <= 1.0) frac = f;

@@ -23,7 +23,7 @@
 //           used entirely.  The row's exact fp16 threshold tau_i (smallest
 //           magnitude whose product with |v_i| reaches c) turns the product
 //           rule into a magnitude compare.  Rows with k_i * H >= f * n (f the
-//           dense fraction, 0.3 by default) are "dense" (read from the dense
+//           dense fraction, 0.2 by default) are "dense" (read from the dense
 //           copy), other active rows are "sparse" (read from the sorted
 //           buckets), rows whose largest product is below c are off.  Records
 //           {v_i, tau_i, row} of a 32-row group are written sparse rows first,
