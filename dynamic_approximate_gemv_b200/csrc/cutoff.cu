@@ -199,8 +199,10 @@ __global__ void __launch_bounds__(kCutThreads, 1) k_cutoff_dispatch(const __grid
 
   int mode = jb.mode;
   if (threadIdx.x == 0) cs.ncand = 0u;
-  // the first-pass histogram and this CTA's merged slice, zeroed while the
-  // chart's loads are in flight (the barrier after the chart covers both)
+  // the first-pass histogram and this CTA's merged slice, zeroed first: the
+  // block barrier after the chart orders the histogram's zeroing before its
+  // atomics, the split cluster barrier below orders the slice's zeroing
+  // before other CTAs add into it
   const int per = kBins0 / cl;
   unsigned* own = mg0;  // this CTA's merged slice lives at the start of the shared area
   if (mode == kModeSelect) {
