@@ -310,9 +310,3 @@ def effort_gemv_batched(preps, hidx, vidx, V, efforts):
 def dense_gemv(W_bits: np.ndarray, v) -> np.ndarray:
     """Plain out = W^T v in float64 (the dense baseline of the method)."""
     return fp16_bits_to_float64(W_bits).T @ as_f32_vector(v).astype(np.float64)
-
-
-def rms_normalize(y: np.ndarray, eps: float = 1e-5) -> np.ndarray:
-    """y / sqrt(mean(y^2) + eps) in float64, no gain (chained-matvec harness)."""
-    y = np.asarray(y, dtype=np.float64)
-    return y / math.sqrt(float(np.mean(y * y)) + eps)
