@@ -282,14 +282,6 @@ def effort_gemv(prep: Prepared, v, effort: float) -> Result:
     return Result(c, K, mask, out)
 
 
-def effort_gemv_at_cutoff(prep: Prepared, v, c) -> Result:
-    """The selection and sum for a given cutoff c (used to judge a GPU run
-    by the set its own reported cutoff defines)."""
-    v32 = as_f32_vector(v)
-    mask = selected_mask(prep, v32, np.float32(c))
-    return Result(np.float32(c), -1, mask, approx_mul(prep, v32, mask))
-
-
 def row_prefix_lengths(prep: Prepared, mask: np.ndarray) -> np.ndarray:
     """L_i and a check that row i's used set is the first L_i of its order.
 
@@ -300,11 +292,6 @@ def row_prefix_lengths(prep: Prepared, mask: np.ndarray) -> np.ndarray:
     ranks = np.arange(prep.out_dim)[None, :]
     assert np.array_equal(in_order, ranks < L[:, None]), "used set is not a prefix"
     return L.astype(np.int64)
-
-
-def effort_gemv_batched(preps, hidx, vidx, V, efforts):
-    """Independent matvecs: pair p uses preps[hidx[p]], V[vidx[p]], efforts[p]."""
-    return [effort_gemv(preps[h], V[vi], e) for h, vi, e in zip(hidx, vidx, efforts)]
 
 
 def dense_gemv(W_bits: np.ndarray, v) -> np.ndarray:
