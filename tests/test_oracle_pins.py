@@ -210,6 +210,16 @@ def test_effort_one_non_square_orientation():
     np.testing.assert_allclose(r.out, exact_dense(W, v), rtol=1e-13, atol=1e-15)
 
 
+@pytest.mark.parametrize("seed,I,Od", [(4, 11, 17), (5, 1, 9), (6, 23, 3)])
+def test_dense_gemv_against_exact_rational(seed, I, Od):
+    # the dense baseline W^T v of the method, on non-square shapes (a
+    # transposed operand or a dropped row fails), fp32 and fp16 v
+    W, v = small_problem(seed, I, Od)
+    np.testing.assert_allclose(O.dense_gemv(W, v), exact_dense(W, v), rtol=1e-13, atol=1e-15)
+    v16 = v.astype(np.float16)
+    np.testing.assert_allclose(O.dense_gemv(W, v16), exact_dense(W, v16.astype(np.float32)), rtol=1e-13, atol=1e-15)
+
+
 def test_keep_closed_form_effort_one():
     W, v = small_problem(3, 9, 16)
     keep = 0.75
