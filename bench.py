@@ -36,7 +36,6 @@ N_MATS, N_VECS, GRAPH_STEPS = 10, 8, 40
 SWEEP = (1.0, 0.5, 0.4, 0.25, 0.15)
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
-CPU_SAMPLE_ROWS = 256
 
 
 def args_parse():
@@ -70,66 +69,168 @@ def workload_config():
 
 
 # ----------------------------------------------------------------- CPU oracle
-def oracle_sample(rows=CPU_SAMPLE_ROWS, seed=4):
-    """A `rows`-row slice of the headline workload, prepared for the oracle."""
+def host_info():
+    """The host the CPU numbers come from: usable cores, CPU model, memory."""
+    nproc = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    model = None
+    try:
+        out = subprocess.run(["lscpu"], capture_output=True, text=True, timeout=10).stdout
+        for line in out.splitlines():
+            if line.strip().startswith("Model name:"):
+                model = line.split(":", 1)[1].strip()
+                break
+    except Exception:
+        pass
+    if not model:
+        try:
+            with open("/proc/cpuinfo") as f:
+                for line in f:
+                    if line.startswith("model name"):
+                        model = line.split(":", 1)[1].strip()
+                        break
+        except Exception:
+            pass
+    mem_gb = None
+    try:
+        with open("/proc/meminfo") as f:
+            for line in f:
+                if line.startswith("MemAvailable:"):
+                    mem_gb = int(line.split()[1]) / 1e6
+    except Exception:
+        pass
+    return {"nproc": nproc, "cpu_model": model, "mem_available_gb": mem_gb}
+
+
+def oracle_workload(rows=IN_DIM, seed=4, n_vecs=4):
+    """The headline workload (or its first `rows` rows) prepared for the oracle
+    (the offline step, not timed) and a few of its vectors."""
     from dynamic_approximate_gemv_b200 import inputs
     from oracle import effort_oracle as O
     Wn = inputs.weights(rows, OUT_DIM, seed)
     prep = O.Prepared(Wn.view(np.uint16), KEEP)
-    vs = [inputs.vector(rows, 50 + k, "t3") for k in range(4)]
-    return prep, vs
+    vs = [inputs.vector(rows, 50 + k, "t3") for k in range(n_vecs)]
+    return Wn, prep, vs
 
 
-def time_oracle(steps, warmup, min_seconds=0.0, rows=CPU_SAMPLE_ROWS):
-    """Oracle matvecs on a `rows`-row slice; returns us per full matvec (time
-    scaled by in_dim / rows), the matvecs done and the seconds they took."""
+def time_oracle_calls(prep, vs, min_calls, budget_s=0.0):
+    """Whole oracle matvecs (chart, cutoff, selection, float64 sum) back to back;
+    returns seconds per call, calls and seconds."""
     from oracle import effort_oracle as O
-    prep, vs = oracle_sample(rows)
-    for k in range(warmup):
-        O.effort_gemv(prep, vs[k % len(vs)], EFFORT)
     t0 = time.perf_counter()
-    done = 0
-    while done < steps or (time.perf_counter() - t0) < min_seconds:
-        O.effort_gemv(prep, vs[done % len(vs)], EFFORT)
-        done += 1
+    n = 0
+    while n < min_calls or (time.perf_counter() - t0) < budget_s:
+        O.effort_gemv(prep, vs[n % len(vs)], EFFORT)
+        n += 1
     dt = time.perf_counter() - t0
-    scale = IN_DIM / rows
-    return dt / done * scale * 1e6, done, dt
+    return (dt / n if n else 0.0), n, dt
 
 
-def cpu_baseline_record(us, done, dt, rows=CPU_SAMPLE_ROWS):
-    return {"value": us, "unit": "us", "cores": 1, "kind": "oracle",
-            "sample": f"{done} oracle matvecs on a {rows}x{OUT_DIM} row slice of the workload "
-                      f"({dt:.1f} s), time scaled by {IN_DIM / rows:g} to the full matvec; "
-                      f"numpy, single thread"}
-
-
-REFERENCE_BUDGET_S = 90.0  # the reference arm's timed oracle work, whatever --steps is
-
-
-def reference_rows(steps):
-    """Row-slice size for the reference arm: each of the `steps` timed steps is
-    a bounded sample, so that the whole run takes about REFERENCE_BUDGET_S."""
+def _oracle_worker(args):
+    """One process of the all-core measurement: prepares its own copy of the
+    workload, then times `calls` whole matvecs (wall-clock start and end)."""
+    seed, calls = args
+    sys.path.insert(0, ROOT)
+    _, prep, vs = oracle_workload(seed=seed)
     from oracle import effort_oracle as O
-    prep, vs = oracle_sample(32)
+    t0 = time.time()
+    for k in range(calls):
+        O.effort_gemv(prep, vs[k % len(vs)], EFFORT)
+    return t0, time.time(), calls
+
+
+def cpu_baseline(budget_s=12.0):
+    """The oracle on the host cores: whole matvecs of the headline workload on
+    one thread, the same on all cores (independent processes, one matvec each
+    at a time), and a plain CPU dense GEMV (numpy float32 W^T v through its BLAS,
+    and the oracle's float64 dense product) beside them."""
+    import multiprocessing as mp
+    info = host_info()
+    Wn, prep, vs = oracle_workload()
+    time_oracle_calls(prep, vs, 1)  # warm
+    sec, n, dt = time_oracle_calls(prep, vs, 2, budget_s)
+    # all cores: as many processes as memory allows (a prepared copy and one
+    # call's temporaries take about 6 GB)
+    procs = max(1, int(info["nproc"] or 1))
+    if info["mem_available_gb"]:
+        procs = min(procs, int(info["mem_available_gb"] // 8))
+    procs = max(1, min(procs, 16))
+    allc = None
+    if procs > 1:
+        ctx = mp.get_context("spawn")
+        with ctx.Pool(procs) as pool:
+            res = pool.map(_oracle_worker, [(4, 2)] * procs)
+        t_start = min(r[0] for r in res)
+        t_end = max(r[1] for r in res)
+        calls = sum(r[2] for r in res)
+        allc = {"processes": procs, "matvecs": calls, "seconds": t_end - t_start,
+                "us_per_matvec": (t_end - t_start) / calls * 1e6}
+    # plain dense GEMV on the CPU
+    from oracle import effort_oracle as O
+    W32 = Wn.astype(np.float32)
+    v32 = vs[0].astype(np.float32)
+    W32.T @ v32
+    reps = 20
     t0 = time.perf_counter()
-    O.effort_gemv(prep, vs[0], EFFORT)
-    t32 = max(time.perf_counter() - t0, 1e-4)
-    rows = int(32 * REFERENCE_BUDGET_S / (max(steps, 1) * t32))
-    return max(16, min(CPU_SAMPLE_ROWS, rows // 16 * 16))
+    for _ in range(reps):
+        W32.T @ v32
+    sgemv_us = (time.perf_counter() - t0) / reps * 1e6
+    try:
+        from threadpoolctl import threadpool_info
+        blas_threads = max([d.get("num_threads", 1) for d in threadpool_info()] or [1])
+    except Exception:
+        blas_threads = None
+    t0 = time.perf_counter()
+    O.dense_gemv(Wn.view(np.uint16), vs[0])
+    f64_us = (time.perf_counter() - t0) * 1e6
+    return {"value": sec * 1e6, "unit": "us", "cores": 1, "kind": "oracle",
+            "sample": f"{n} whole oracle matvecs of the {IN_DIM}x{OUT_DIM} workload ({dt:.1f} s), numpy, one "
+                      f"thread (the oracle's own preparation of the matrix is the offline step, not timed)",
+            "all_cores": allc, "host": info,
+            "cpu_dense_gemv": {"numpy_f32_us": sgemv_us, "blas_threads": blas_threads,
+                               "oracle_f64_us": f64_us}}
+
+
+REFERENCE_BUDGET_S = 120.0  # the reference arm's oracle work, whatever --steps is
 
 
 def run_reference(a):
+    """The reference arm: the oracle, as it stands, on the host cores.  Each
+    step is one whole oracle matvec of the workload when all --steps + warmup
+    steps fit in REFERENCE_BUDGET_S; otherwise each step is the oracle on a
+    row slice of the workload, the time per matvec is scaled to the full
+    matrix, and the line says so (`extrapolated`).  ms_per_step is always the
+    time a step really took."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    rows = reference_rows(a.steps)
-    us, done, dt = time_oracle(a.steps, min(a.warmup, 2), rows=rows)
-    line = {"metric": METRIC, "value": us, "unit": "us", "n_gpus": a.gpus, "steps": a.steps, "warmup": a.warmup,
-            "ms_per_step": us / 1000.0, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+    info = host_info()
+    Wn, prep, vs = oracle_workload()
+    sec_full, _, _ = time_oracle_calls(prep, vs, 1)
+    warm = min(a.warmup, 1)
+    if (a.steps + warm) * sec_full <= REFERENCE_BUDGET_S:
+        time_oracle_calls(prep, vs, warm)
+        sec, n, dt = time_oracle_calls(prep, vs, a.steps)
+        value, step_ms, extra = sec * 1e6, sec * 1e3, None
+        sample = f"{n} whole oracle matvecs of the {IN_DIM}x{OUT_DIM} workload ({dt:.1f} s), numpy, one thread"
+    else:
+        del prep
+        rows = int(IN_DIM * REFERENCE_BUDGET_S / ((a.steps + warm) * sec_full))
+        rows = max(16, min(IN_DIM, rows // 16 * 16))
+        _, sprep, svs = oracle_workload(rows=rows)
+        time_oracle_calls(sprep, svs, warm)
+        sec, n, dt = time_oracle_calls(sprep, svs, a.steps)
+        value, step_ms = sec * IN_DIM / rows * 1e6, sec * 1e3
+        extra = {"rows_per_step": rows, "scale_to_full_matvec": IN_DIM / rows,
+                 "whole_matvec_us_measured_once": sec_full * 1e6}
+        sample = (f"{n} oracle matvecs on a {rows}x{OUT_DIM} row slice of the workload ({dt:.1f} s), time per "
+                  f"matvec scaled by {IN_DIM / rows:g} to the full matrix; numpy, one thread")
+    line = {"metric": METRIC, "value": value, "unit": "us", "n_gpus": a.gpus, "steps": a.steps, "warmup": a.warmup,
+            "ms_per_step": step_ms, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
             "dtype": "f64", "data": "synthetic", "impl": "reference", "config": workload_config(),
-            "cpu_baseline": cpu_baseline_record(us, done, dt, rows),
-            "e2e": {"value": us, "unit": "us", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+            "cpu_baseline": {"value": value, "unit": "us", "cores": 1, "kind": "oracle", "sample": sample,
+                             "host": info},
+            "extrapolated": extra,
+            "e2e": {"value": value, "unit": "us", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
@@ -531,50 +632,15 @@ def main():
     us_per_step = ms * 1000.0 / a.steps
     value = whole_job_us_per_matvec(us_per_step, world)
 
-    # per-kernel durations: the split call records an event between the two
-    # kernels; the calls are captured in a CUDA graph (external event-record
-    # nodes) so that host launch gaps do not enter the kernel times
-    n_ph = GRAPH_STEPS
-    s = torch.cuda.Stream(device=dev)
-    evA = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n_ph + 1)]
-    evB = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n_ph)]
-    for ev in evA + evB:
-        ev.record(s)  # creates the CUDA events
-    torch.cuda.synchronize()
-
-    def phase_calls():
-        for k, (mi, vi) in enumerate(step_pairs(n_ph)):
-            evA[k].record(s)
-            mats[mi].gemv_split(vecs[vi], EFFORT, outs[mi], evB[k], stream=s)
-        evA[n_ph].record(s)
-
-    s.wait_stream(torch.cuda.current_stream(dev))
-    with torch.cuda.stream(s):
-        phase_calls()  # warm once outside capture
-    torch.cuda.synchronize()
-    gph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(gph, stream=s):
-        phase_calls()
-    torch.cuda.synchronize()
-    cut_ms, mac_ms = [], []
-    for rep in range(8):
-        gph.replay()
-        torch.cuda.synchronize()
-        if rep >= 3:
-            cut_ms += [evA[k].elapsed_time(evB[k]) for k in range(n_ph)]
-            mac_ms += [evB[k].elapsed_time(evA[k + 1]) for k in range(n_ph)]
-    mac_us = statistics.mean(mac_ms) * 1000.0
-    cut_us = statistics.mean(cut_ms) * 1000.0
-    del gph
-
     S_mean = mean_count(EFFORT)
-    alg_bytes = 3.0 * S_mean + 4.0 * IN_DIM + 4.0 * OUT_DIM  # F3 bytes of the used set + v + out
-    achieved = alg_bytes / (mac_us * 1e-6) / 1e9
-    traffic = ncu_traffic("k_mac")
+    alg_bytes = 3.0 * S_mean + 4.0 * IN_DIM + 4.0 * OUT_DIM  # 3-byte entries of the used set + v + out
+    launch_us = us_per_step  # one kernel per call
+    achieved = alg_bytes / (launch_us * 1e-6) / 1e9
+    traffic = ncu_traffic("k_effort")
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                "traffic": traffic, "kernel": "k_mac", "peak_kind": peak_kind,
+                "traffic": traffic, "kernel": "k_effort", "peak_kind": peak_kind,
                 "frac_of_nominal_8000": achieved / NOMINAL_HBM_GBS,
-                "algorithmic_bytes_per_launch": alg_bytes, "launch_us": mac_us}
+                "algorithmic_bytes_per_launch": alg_bytes, "launch_us": launch_us}
 
     # dense baselines on the same rotation (raw fp16 matrices, 117 MB each)
     ws = E.Workspace(IN_DIM, OUT_DIM)
@@ -690,8 +756,7 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
-        us_o, done, dt = time_oracle(2, 1, min_seconds=10.0)
-        cpu = cpu_baseline_record(us_o, done, dt)
+        cpu = cpu_baseline()
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": "us", "n_gpus": world, "steps": a.steps,
@@ -702,8 +767,7 @@ def main():
                 "roofline": roofline, "cpu_baseline": cpu,
                 "e2e": {"value": e2e_us, "unit": "us", "h2d_bytes_per_step": 4 * IN_DIM,
                         "d2h_bytes_per_step": 4 * OUT_DIM},
-                "gpu_launches": 2 * a.steps, "clocks": clocks,
-                "phases_us": {"cutoff_dispatch": cut_us, "mac": mac_us},
+                "gpu_launches": a.steps, "clocks": clocks,
                 "mean_used_products": S_mean, "baselines": baselines, "sweep": sweep,
                 "shapes": shapes,
                 "chain": chain,

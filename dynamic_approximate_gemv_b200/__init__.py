@@ -17,6 +17,9 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libeffort.so")
+# EFFORT_DEBUG_LIB=1 loads the bounds-checking build (kernels compiled with
+# -DEFFORT_DEBUG report bad indices through effort_check instead of using them)
+LIB_DEBUG_PATH = os.path.join(_HERE, "libeffort_debug.so")
 
 F32, F16 = 0, 1
 STATUS = {0: "ok", 1: "invalid argument", 2: "CUDA error", 3: "out of memory",
@@ -35,27 +38,30 @@ class EffortError(RuntimeError):
 
 class Layout(ctypes.Structure):
     _fields_ = [("in_dim", ctypes.c_int64), ("out_dim", ctypes.c_int64),
-                ("n_kept", ctypes.c_int32), ("n_tiles", ctypes.c_int32), ("bucket_cap", ctypes.c_int32),
-                ("ck_step", ctypes.c_int32), ("n_ck", ctypes.c_int32), ("n_probes", ctypes.c_int32),
-                ("vals", ctypes.c_void_p), ("idx", ctypes.c_void_p), ("probes", ctypes.c_void_p),
-                ("ckmag", ctypes.c_void_p), ("cnt", ctypes.c_void_p), ("wdense", ctypes.c_void_p),
-                ("rec", ctypes.c_void_p), ("gcnt", ctypes.c_void_p), ("n_groups", ctypes.c_int32)]
+                ("n_kept", ctypes.c_int32), ("n_panels", ctypes.c_int32), ("panel_width", ctypes.c_int32),
+                ("chunk_slots", ctypes.c_int32), ("store_num", ctypes.c_int32), ("store_den", ctypes.c_int32),
+                ("n_probes", ctypes.c_int32), ("dense_stride", ctypes.c_int32), ("total_chunks", ctypes.c_uint32),
+                ("vals", ctypes.c_void_p), ("gaps", ctypes.c_void_p), ("head", ctypes.c_void_p),
+                ("lists", ctypes.c_void_p), ("wdense", ctypes.c_void_p), ("probes", ctypes.c_void_p),
+                ("scratch_bytes", ctypes.c_size_t)]
 
 
 def lib():
     """Load libeffort.so (built in-tree by dynamic_approximate_gemv_b200.build)."""
     global _lib
     if _lib is None:
-        if not os.path.exists(LIB_PATH):
-            raise RuntimeError(f"{LIB_PATH} is missing: run `python -m dynamic_approximate_gemv_b200.build`")
-        L = ctypes.CDLL(LIB_PATH)
+        path = LIB_DEBUG_PATH if os.environ.get("EFFORT_DEBUG_LIB") == "1" else LIB_PATH
+        if not os.path.exists(path):
+            raise RuntimeError(f"{path} is missing: run `python -m dynamic_approximate_gemv_b200.build`")
+        L = ctypes.CDLL(path)
         vp, i64, i32, f32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float
         sig = {
             "effort_prepare": [vp, i64, i64, f32, vp, ctypes.POINTER(vp)],
             "effort_gemv": [vp, vp, f32, vp, vp],
             "effort_gemv_ex": [vp, vp, ctypes.c_int, f32, vp, vp, vp, vp, vp],
-            "effort_gemv_split": [vp, vp, ctypes.c_int, f32, vp, vp, vp, vp, vp],
             "effort_gemv_host": [vp, vp, ctypes.c_int, f32, vp, vp],
+            "effort_gemv_timed": [vp, vp, ctypes.c_int, f32, vp, vp, vp],
+            "effort_grid_blocks": [vp, ctypes.POINTER(i32)],
             "effort_gemv_static": [vp, vp, ctypes.c_int, f32, vp, vp, vp, vp, vp],
             "effort_check": [vp],
             "effort_workspace_create": [i64, i64, i32, ctypes.POINTER(vp)],
@@ -66,6 +72,8 @@ def lib():
                                 ctypes.POINTER(ctypes.c_size_t)],
             "effort_get_layout": [vp, ctypes.POINTER(Layout)],
             "effort_destroy": [vp],
+            "effort_device_bytes_held": [ctypes.POINTER(ctypes.c_uint64)],
+            "effort_last_call_bytes": [vp, ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(ctypes.c_uint64)],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -190,18 +198,29 @@ class PreparedMatrix:
                "effort_gemv_static")
         return out
 
-    def gemv_split(self, v, effort, out, mid_event, stream=None):
-        """gemv that records `mid_event` (a recorded-once torch.cuda.Event) between the
-        cutoff/dispatch kernel and the multiply kernel, for per-phase timing."""
+    def grid_blocks(self):
+        n = ctypes.c_int32()
+        _check(lib().effort_grid_blocks(self._h, ctypes.byref(n)), "effort_grid_blocks")
+        return n.value
+
+    def gemv_timed(self, v, effort, out, marks):
+        """gemv that stores per-phase global-timer marks into `marks`
+        (int64 [grid_blocks(), 16] on the device)."""
         _need_cuda(v, "v")
         _need_cuda(out, "out")
-        if not mid_event.cuda_event:
-            raise ValueError("mid_event has no CUDA event yet: record it once first")
-        st = stream if stream is not None else torch.cuda.current_stream(v.device)
-        _check(lib().effort_gemv_split(self._h, _ptr(v), _vdtype(v), ctypes.c_float(effort), _ptr(out), None, None,
-                                       ctypes.c_void_p(mid_event.cuda_event), ctypes.c_void_p(st.cuda_stream)),
-               "effort_gemv_split")
+        _need_cuda(marks, "marks")
+        if marks.dtype != torch.int64 or tuple(marks.shape) != (self.grid_blocks(), 16):
+            raise ValueError("marks must be int64 [grid_blocks(), 16]")
+        _check(lib().effort_gemv_timed(self._h, _ptr(v), _vdtype(v), ctypes.c_float(effort), _ptr(out), _ptr(marks),
+                                       _stream(v.device)), "effort_gemv_timed")
         return out
+
+    def last_call_bytes(self):
+        """(dense, sparse) bytes of the prepared matrix the last finished call
+        planned to read (synchronises the handle's stream)."""
+        d, sp = ctypes.c_uint64(), ctypes.c_uint64()
+        _check(lib().effort_last_call_bytes(self._h, ctypes.byref(d), ctypes.byref(sp)), "effort_last_call_bytes")
+        return d.value, sp.value
 
     def check(self):
         _check(lib().effort_check(self._h), "effort_check")
@@ -217,17 +236,18 @@ class PreparedMatrix:
         """Device storage as read-only torch views (for format checks)."""
         L = Layout()
         _check(lib().effort_get_layout(self._h, ctypes.byref(L)), "effort_get_layout")
-        I, T, cap, C = L.in_dim, L.n_tiles, L.bucket_cap, L.n_ck
+        I, P, nc, cs = L.in_dim, L.n_panels, L.total_chunks, L.chunk_slots
 
         def view(ptr, shape, typestr):
             return torch.as_tensor(_CudaView(ptr, shape, typestr), device=self.device)
 
         return {
-            "n_kept": L.n_kept, "n_tiles": T, "bucket_cap": cap, "ck_step": L.ck_step, "n_ck": C,
-            "vals": view(L.vals, (T, I, cap), "<i2"), "idx": view(L.idx, (T, I, cap), "|u1"),
-            "probes": view(L.probes, (I, L.n_probes), "<i2"), "ckmag": view(L.ckmag, (I, C + 1), "<i2"),
-            "cnt": view(L.cnt, (I, C, T), "|u1"), "wdense": view(L.wdense, (I, T * 256), "<i2"),
-            "rec": view(L.rec, (L.n_groups, 32, 2), "<u4"), "gcnt": view(L.gcnt, (L.n_groups,), "<u4"),
+            "n_kept": L.n_kept, "n_panels": P, "panel_width": L.panel_width, "chunk_slots": cs,
+            "store_num": L.store_num, "store_den": L.store_den, "total_chunks": nc,
+            "dense_stride": L.dense_stride, "scratch_bytes": L.scratch_bytes,
+            "vals": view(L.vals, (max(nc, 1) * cs,), "<i2"), "gaps": view(L.gaps, (max(nc, 1) * cs,), "|u1"),
+            "head": view(L.head, (max(nc, 1),), "<i2"), "lists": view(L.lists, (I, P, 4), "<u4"),
+            "wdense": view(L.wdense, (I, L.dense_stride), "<i2"), "probes": view(L.probes, (I, L.n_probes), "<i2"),
         }
 
     def close(self):
@@ -263,6 +283,13 @@ class Workspace:
             self.close()
         except Exception:
             pass
+
+
+def device_bytes_held():
+    """Device memory the library holds now (all handles and workspaces)."""
+    x = ctypes.c_uint64()
+    _check(lib().effort_device_bytes_held(ctypes.byref(x)), "effort_device_bytes_held")
+    return x.value
 
 
 def gemv_batched(ws, mats, hidx, vidx, V, efforts, OUT=None, cutoffs=None, counts=None):

@@ -1,153 +1,151 @@
 // Host side of the C ABI declared in include/effort.h: argument checks,
 // storage and scratch allocation, the host arithmetic of each call (the
 // target count K, the call mode) and the kernel launches.  Every step of the
-// matvec itself runs in the kernels of prep.cu, cutoff.cu, mac.cu, dense.cu.
+// matvec itself runs in the kernels of prep.cu, effort.cu and dense.cu.
 #include <math.h>
 #include <stdlib.h>
 #include <string.h>
 
+#include <atomic>
 #include <new>
 
 #include "../../include/effort.h"
 #include "effort_internal.cuh"
 
 namespace effort {
-cudaError_t launch_prep(const uint16_t* W, const HandleDesc* d_desc, int I, int O, uint16_t* vals, uint8_t* idx,
-                        uint16_t* wdense, uint16_t* probes, uint16_t* ckmag, uint8_t* cnt, unsigned int* status,
-                        cudaStream_t stream);
-cudaError_t launch_cutoff(const Jobs<1>& jobs, int I, int cl, cudaStream_t stream);
-cudaError_t launch_cutoff_batch(const Jobs<kMaxJobs>& jobs, int njobs, int I, int cl, cudaStream_t stream);
-cudaError_t launch_mac(const Jobs<1>& jobs, int T, int S, cudaStream_t stream);
-cudaError_t launch_mac_batch(const Jobs<kMaxJobs>& jobs, int njobs, int T, int S, cudaStream_t stream);
+cudaError_t launch_prep(const uint16_t* W, int I, int O, int n, int P, int dstride, const int* prank,
+                        uint16_t* wdense, uint16_t* probes, uint16_t* vals, uint8_t* gaps, uint16_t* head, uint4* lst,
+                        unsigned* chunk_count, unsigned cap_chunks, unsigned* status, cudaStream_t stream);
+unsigned long long prep_chunk_bound_per_row(int O, int n);
+cudaError_t effort_kernel_attributes(size_t smem);
+int effort_blocks_per_sm(size_t smem);
+cudaError_t launch_effort(const Job& job, int nb, size_t smem, cudaStream_t stream);
 cudaError_t launch_dense(const uint16_t* W, int I, int O, const void* v, int vdtype, float* out, float* part,
                          unsigned* tilecnt, int T, int S, cudaStream_t stream);
-int mac_ctas_per_sm();
 int dense_ctas_per_sm();
-cudaError_t init_kernel_attributes();
-size_t cutoff_max_dynamic_smem();
-int cutoff_max_clusters(int cl, size_t smem);
 }  // namespace effort
 
 using namespace effort;
 
 namespace {
 
-struct Geometry {
-  int I, O, T, G;
-  int S;        // row slices of the multiply kernel (grid T x S)
-  int S_dense;  // row slices of the dense baseline
-  int cl;       // CTAs in the cutoff cluster
-  int dense_q16;  // dense-row threshold (share of the row surely used, x 65536)
-};
-
-struct WsBlock {
-  void* base = nullptr;
-  size_t bytes = 0;
-  WsPtrs p = {};
-};
-
-int g_num_sms = 0;
-int g_smem_optin = 0;
-
-cudaError_t device_info() {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  e = cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
-  if (e != cudaSuccess) return e;
-  return cudaDeviceGetAttribute(&g_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-}
-
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// Chooses the cutoff cluster size and the split-K slice counts.
-effort_status_t make_geometry(int64_t I, int64_t O, Geometry* g) {
-  if (device_info() != cudaSuccess) return EFFORT_ERR_CUDA;
-  if (init_kernel_attributes() != cudaSuccess) return EFFORT_ERR_CUDA;
+// ---------------------------------------------------------------- allocation
+// Every device allocation of the library goes through dev_alloc.  An optional
+// cap on the bytes the library holds at once (environment variable
+// EFFORT_ALLOC_CAP_BYTES) turns larger requests into EFFORT_ERR_NOMEM before
+// CUDA is asked, which lets allocation failure be exercised on purpose.
+std::atomic<unsigned long long> g_live_bytes{0};
+
+unsigned long long alloc_cap() {
+  const char* e = getenv("EFFORT_ALLOC_CAP_BYTES");
+  if (!e || !*e) return ~0ull;
+  return strtoull(e, nullptr, 10);
+}
+bool within_cap(size_t bytes) { return g_live_bytes.load() + bytes <= alloc_cap(); }
+
+effort_status_t dev_alloc(void** p, size_t bytes) {
+  *p = nullptr;
+  if (!within_cap(bytes)) return EFFORT_ERR_NOMEM;
+  if (cudaMalloc(p, bytes) != cudaSuccess) {
+    cudaGetLastError();
+    *p = nullptr;
+    return EFFORT_ERR_NOMEM;
+  }
+  g_live_bytes += bytes;
+  return EFFORT_OK;
+}
+void dev_free(void* p, size_t bytes) {
+  if (!p) return;
+  cudaFree(p);
+  g_live_bytes -= bytes;
+}
+
+struct DevBuf {
+  void* p = nullptr;
+  size_t bytes = 0;
+  effort_status_t alloc(size_t b) {
+    bytes = b;
+    return dev_alloc(&p, b);
+  }
+  void release() {
+    dev_free(p, bytes);
+    p = nullptr;
+    bytes = 0;
+  }
+};
+
+// ---------------------------------------------------------------- geometry
+struct Geometry {
+  int I, O, n, P, dstride;
+  int nb;       // blocks of the matvec kernel (one per SM)
+  size_t smem;  // its dynamic shared memory
+  int T;        // 256-column tiles (dense baseline)
+  int S_dense;  // row slices of the dense baseline
+};
+
+effort_status_t make_geometry(int64_t I, int64_t O, int n, Geometry* g) {
+  int dev = 0, sms = 0, optin = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return EFFORT_ERR_CUDA;
+  }
   g->I = (int)I;
   g->O = (int)O;
-  g->T = (int)((O + kTW - 1) / kTW);
-  g->G = (int)((I + kGroupRows - 1) / kGroupRows);
-  g->cl = 0;
-  const size_t dyn_max = cutoff_max_dynamic_smem();
-  for (int cl : {16, 8}) {  // the wider cluster halves each CTA's share of the rows
-    const size_t sm = cut_smem_bytes(g->I, cl);
-    if (sm <= dyn_max && cutoff_max_clusters(cl, sm) >= 1) {
-      g->cl = cl;
-      break;
-    }
+  g->n = n;
+  g->P = (int)((O + kPW - 1) / kPW);
+  g->dstride = (int)((O + kStripe - 1) / kStripe * kStripe);
+  g->T = (int)((O + 255) / 256);
+  size_t oc, oh, ocd, ol, octl;
+  g->nb = sms;
+  g->smem = smem_layout(g->I, g->nb, &oc, &oh, &ocd, &ol, &octl);
+  if (g->smem > (size_t)optin) return EFFORT_ERR_UNSUPPORTED;
+  if (effort_kernel_attributes(g->smem) != cudaSuccess) {
+    cudaGetLastError();
+    return EFFORT_ERR_CUDA;
   }
-  if (g->cl == 0) return EFFORT_ERR_UNSUPPORTED;
-  // T x S CTAs fill the SMs once (two resident per SM); every slice keeps at
-  // least one 32-row group
-  const int slots = g_num_sms * mac_ctas_per_sm();
-  int S = slots / g->T;
-  if (S < 1) S = 1;
-  if (S > g->G) S = g->G;
-  g->S = S;
-  // rows whose surely-used share reaches this fraction are read from the dense
-  // copy (2 B per weight, register accumulation) instead of their buckets.  A
-  // sparse row-tile's short prefix rounds up to whole sectors twice (values,
-  // columns), so a row read through its buckets costs more per used product
-  // than its byte count suggests; measured step times are flat from 0.1 to
-  // 0.2 and rise above that
-  double frac = 0.2;
-  if (const char* env = getenv("EFFORT_DENSE_FRACTION")) {
-    const double f = atof(env);
-    if (f > 0.0 && f <= 1.0) frac = f;
-  }
-  g->dense_q16 = (int)(frac * 65536.0 + 0.5);
-  // the dense baseline's T x Sd CTAs fill the SMs once as well
-  int Sd = (g_num_sms * dense_ctas_per_sm()) / g->T;
+  if (effort_blocks_per_sm(g->smem) < 1) return EFFORT_ERR_UNSUPPORTED;
+  int Sd = (sms * dense_ctas_per_sm()) / g->T;
   if (Sd < 1) Sd = 1;
   if (Sd > (int)((I + 7) / 8)) Sd = (int)((I + 7) / 8);
-  if (Sd < 1) Sd = 1;
-  g->S_dense = Sd;
+  g->S_dense = Sd < 1 ? 1 : Sd;
   return EFFORT_OK;
 }
 
-// One contiguous device block of scratch for `npairs` jobs.
-effort_status_t alloc_ws(const Geometry& g, int npairs, WsBlock* out, WsPtrs* slots) {
-  const int S = g.S > g.S_dense ? g.S : g.S_dense;
-  const size_t per = align_up(256, 256)                                  // c, count, done, status
-                     + align_up((size_t)g.T * 4, 256)                    // tilecnt
-                     + align_up((size_t)g.G * 4, 256)                    // gcnt
-                     + align_up((size_t)g.G * g.T * 32, 256)             // ut
-                     + align_up((size_t)g.G * kRecPerGroup * 8, 256)     // rec
-                     + align_up((size_t)S * g.T * kTW * 4, 256);         // part
-  const size_t bytes = per * (size_t)npairs;
-  void* base = nullptr;
-  if (cudaMalloc(&base, bytes) != cudaSuccess) {
-    cudaGetLastError();
-    return EFFORT_ERR_NOMEM;
-  }
-  if (cudaMemset(base, 0, bytes) != cudaSuccess) {
-    cudaFree(base);
-    return EFFORT_ERR_CUDA;
-  }
-  for (int p = 0; p < npairs; ++p) {
-    char* b = (char*)base + per * p;
-    WsPtrs w;
-    w.c = (float*)(b + 0);
-    w.count = (unsigned long long*)(b + 8);
-    w.done = (unsigned int*)(b + 16);
-    w.status = (unsigned int*)(b + 20);
-    b += 256;
-    w.tilecnt = (unsigned int*)b;
-    b += align_up((size_t)g.T * 4, 256);
-    w.gcnt = (unsigned int*)b;
-    b += align_up((size_t)g.G * 4, 256);
-    w.ut = (unsigned char*)b;
-    b += align_up((size_t)g.G * g.T * 32, 256);
-    w.rec = (uint2*)b;
-    b += align_up((size_t)g.G * kRecPerGroup * 8, 256);
-    w.part = (float*)b;
-    slots[p] = w;
-  }
-  out->base = base;
-  out->bytes = bytes;
-  out->p = slots[0];
-  return EFFORT_OK;
+// ---------------------------------------------------------------- scratch
+// Bytes of one call's scratch, carved in this order.
+size_t scratch_bytes(const Geometry& g) {
+  return align_up((size_t)kHdrWords * 4 + 16, 256)                 // header, barrier, count
+         + align_up((size_t)(kBins0 + kBins1 + kBins2) * 4, 256)   // histograms
+         + align_up((size_t)kCandCap * 8, 256)                     // candidates
+         + 2 * align_up((size_t)g.I * g.P * 4, 256)                // info, rowpre
+         + align_up((size_t)g.nb * g.P * 4, 256);                  // block totals
+}
+// Bytes that must be zero before the first call (header and histograms).
+size_t scratch_zero_bytes() {
+  return align_up((size_t)kHdrWords * 4 + 16, 256) + align_up((size_t)(kBins0 + kBins1 + kBins2) * 4, 256);
+}
+
+WsPtrs carve(char* b, const Geometry& g) {
+  WsPtrs w;
+  w.hdr = (unsigned*)b;
+  w.bar = (unsigned long long*)(b + kHdrWords * 4);
+  w.count = w.bar + 1;
+  b += align_up((size_t)kHdrWords * 4 + 16, 256);
+  w.ghist0 = (unsigned*)b;
+  w.ghist1 = w.ghist0 + kBins0;
+  w.ghist2 = w.ghist1 + kBins1;
+  b += align_up((size_t)(kBins0 + kBins1 + kBins2) * 4, 256);
+  w.cand = (uint2*)b;
+  b += align_up((size_t)kCandCap * 8, 256);
+  w.info = (unsigned*)b;
+  b += align_up((size_t)g.I * g.P * 4, 256);
+  w.rowpre = (unsigned*)b;
+  b += align_up((size_t)g.I * g.P * 4, 256);
+  w.ctot = (unsigned*)b;
+  return w;
 }
 
 unsigned long long target_count(float effort, long long N) {
@@ -190,12 +188,12 @@ struct effort_handle_s {
   Geometry g = {};
   float keep = 1.0f;
   HandleDesc hd = {};
-  HandleDesc* d_desc = nullptr;
-  void* storage = nullptr;
-  size_t storage_bytes = 0;
-  WsBlock ws;
+  DevBuf chunks;   // vals, gaps, head
+  DevBuf tables;   // lst, wdense, probes
+  DevBuf ws;       // per-call scratch
+  DevBuf stage;    // effort_gemv_host staging: v (in_dim x 4 B), then out (out_dim x 4 B)
   WsPtrs slot = {};
-  void* stage = nullptr;  // device staging of effort_gemv_host: v (in_dim x 4 B), then out (out_dim x 4 B)
+  size_t storage_bytes = 0;
   cudaStream_t last_stream = nullptr;
 };
 
@@ -203,10 +201,64 @@ struct effort_workspace_s {
   int dev = 0;
   Geometry g = {};
   int max_pairs = 0;
-  WsBlock ws;
-  WsPtrs* slots = nullptr;
+  DevBuf ws;
+  WsPtrs slot = {};
+  DevBuf dense_part;  // dense baseline: partial tiles and arrival counters
   cudaStream_t last_stream = nullptr;
 };
+
+namespace effort {
+
+// The scratch header words, barrier counter and histograms start at zero.
+cudaError_t clear_scratch(const WsPtrs& w, cudaStream_t s) {
+  cudaError_t e = cudaMemsetAsync(w.hdr, 0, align_up((size_t)kHdrWords * 4 + 16, 256), s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(w.ghist0, 0, (size_t)(kBins0 + kBins1 + kBins2) * 4, s);
+  return e;
+}
+
+size_t handle_scratch_bytes(effort_handle_t h) { return scratch_bytes(h->g); }
+WsPtrs handle_carve(effort_handle_t h, char* base) { return carve(base, h->g); }
+size_t handle_scratch_zero_bytes() { return scratch_zero_bytes(); }
+
+static effort_status_t fill_job(effort_handle_t h, const WsPtrs& ws, const void* v, effort_dtype_t v_dtype,
+                                float effort, float* out, float* cutoff_out, uint64_t* count_out,
+                                uint32_t* rowlen_out, Job* j) {
+  if (!v || !out) return EFFORT_ERR_ARG;
+  if (v_dtype != EFFORT_F32 && v_dtype != EFFORT_F16) return EFFORT_ERR_ARG;
+  if (!effort_ok(effort)) return EFFORT_ERR_ARG;
+  const long long N = (long long)h->g.I * (long long)h->g.O;
+  const unsigned long long K = target_count(effort, N);
+  memset(j, 0, sizeof(*j));
+  j->hd = h->hd;
+  j->barrier_nb = (unsigned)h->g.nb;
+  // test hook: a barrier count no grid reaches makes every grid-wide wait run
+  // out (bounded) so that the timeout status and the recovery can be checked
+  if (const char* t = getenv("EFFORT_TEST_UNREACHABLE_BARRIER"))
+    if (t[0] == '1') j->barrier_nb = (unsigned)h->g.nb + 1u;
+  j->v = v;
+  j->out = out;
+  j->cutoff_out = cutoff_out;
+  j->count_out = (unsigned long long*)count_out;
+  j->rowlen_out = rowlen_out;
+  j->ws = ws;
+  j->K = K;
+  j->mode = (K >= h->hd.kept_total) ? kModeAll : (K == 0 ? kModeNone : kModeSelect);
+  j->vdtype = (int)v_dtype;
+  return EFFORT_OK;
+}
+
+effort_status_t handle_fill_job(effort_handle_t h, const WsPtrs& ws, const void* v, effort_dtype_t v_dtype,
+                                float effort, float* out, float* cutoff_out, uint64_t* count_out, Job* j) {
+  if (!h) return EFFORT_ERR_ARG;
+  return fill_job(h, ws, v, v_dtype, effort, out, cutoff_out, count_out, nullptr, j);
+}
+
+cudaError_t handle_launch(effort_handle_t h, const Job& j, cudaStream_t s) {
+  return launch_effort(j, h->g.nb, h->g.smem, s);
+}
+int handle_device(effort_handle_t h) { return h->dev; }
+
+}  // namespace effort
 
 extern "C" {
 
@@ -217,7 +269,7 @@ const char* effort_status_string(effort_status_t s) {
     case EFFORT_ERR_CUDA: return "CUDA error";
     case EFFORT_ERR_NOMEM: return "out of memory";
     case EFFORT_ERR_NONFINITE: return "non-finite input";
-    case EFFORT_ERR_DEVICE: return "device-side inconsistency";
+    case EFFORT_ERR_DEVICE: return "device-side inconsistency or timeout";
     case EFFORT_ERR_UNSUPPORTED: return "unsupported size";
   }
   return "unknown status";
@@ -235,172 +287,142 @@ effort_status_t effort_prepare(const void* W, int64_t in_dim, int64_t out_dim, f
   const int n = (int)floor((double)keep_fraction * (double)out_dim + 0.5);
   if (n < 1) return EFFORT_ERR_ARG;
 
+  // storage sizes need no device: check them against the allocation cap first
+  const int I = (int)in_dim, O = (int)out_dim;
+  const int P = (O + kPW - 1) / kPW, dstride = (O + kStripe - 1) / kStripe * kStripe;
+  const unsigned long long cap_chunks = prep_chunk_bound_per_row(O, n) * (unsigned long long)I;
+  const size_t sz_lst = align_up((size_t)I * P * 16, 256);
+  const size_t sz_dense = align_up((size_t)I * dstride * 2, 256);
+  const size_t sz_probe = align_up((size_t)I * kP * 2, 256);
+  const size_t sz_tables = sz_lst + sz_dense + sz_probe + 256;
+  const size_t sz_tmp = align_up((size_t)cap_chunks * kCS * 3 + (size_t)cap_chunks * 2, 256);
+  if (!within_cap(sz_tables + sz_tmp)) return EFFORT_ERR_NOMEM;
+  if (cap_chunks >= (1ull << 31)) return EFFORT_ERR_UNSUPPORTED;
+
   effort_handle_s* h = new (std::nothrow) effort_handle_s();
   if (!h) return EFFORT_ERR_NOMEM;
-  cudaGetDevice(&h->dev);
-  effort_status_t st = make_geometry(in_dim, out_dim, &h->g);
+  if (cudaGetDevice(&h->dev) != cudaSuccess) {
+    cudaGetLastError();
+    delete h;
+    return EFFORT_ERR_CUDA;
+  }
+  effort_status_t st = make_geometry(in_dim, out_dim, n, &h->g);
   if (st != EFFORT_OK) {
     delete h;
     return st;
   }
   h->keep = keep_fraction;
-  const Geometry& g = h->g;
-  const int I = g.I, T = g.T;
-  int H = 2 * T;
-  H = (H + 31) / 32 * 32;
-  if (H < 32) H = 32;
-  const int C = (n + H - 1) / H;
-
   HandleDesc& d = h->hd;
   d.I = I;
-  d.O = g.O;
-  d.T = T;
+  d.O = O;
   d.n = n;
-  d.C = C;
-  d.H = H;
-  d.dstride = T * kTW;
+  d.P = P;
+  d.dstride = dstride;
   d.kept_total = (unsigned long long)I * (unsigned long long)n;
+  int prank[kP];
   for (int k = 1; k <= kP; ++k) {
     const int b0 = (int)(((long long)(k - 1) * n) / kP), b1 = (int)(((long long)k * n) / kP);
     d.pw[k - 1] = b1 - b0;
-    d.prank[k - 1] = (b1 > b0) ? (b0 + b1) / 2 : -1;
+    prank[k - 1] = (b1 > b0) ? (b0 + b1) / 2 : -1;
   }
 
-  const size_t nb = (size_t)T * I * kCap;
-  const size_t sz_vals = align_up(nb * 2, 256), sz_idx = align_up(nb, 256);
-  const size_t sz_dense = align_up((size_t)I * T * kTW * 2, 256);
-  const size_t sz_probe = align_up((size_t)I * kP * 2, 256);
-  const size_t sz_ck = align_up((size_t)I * (C + 1) * 2, 256);
-  const size_t sz_cnt = align_up((size_t)I * C * T, 256);
-  const size_t sz_desc = align_up(sizeof(HandleDesc), 256);
-  const size_t sz_status = 256;
-  const size_t total = sz_vals + sz_idx + sz_dense + sz_probe + sz_ck + sz_cnt + sz_desc + sz_status;
-  if (cudaMalloc(&h->storage, total) != cudaSuccess) {
+  DevBuf tmp;
+  auto fail = [&](effort_status_t s) {
     cudaGetLastError();
+    tmp.release();
+    h->tables.release();
+    h->chunks.release();
+    h->ws.release();
+    h->stage.release();
     delete h;
-    return EFFORT_ERR_NOMEM;
-  }
-  h->storage_bytes = total;
-  char* b = (char*)h->storage;
-  d.vals = (const uint16_t*)b;
-  b += sz_vals;
-  d.idx = (const uint8_t*)b;
-  b += sz_idx;
-  d.wdense = (const uint16_t*)b;
-  b += sz_dense;
-  d.probes = (const uint16_t*)b;
-  b += sz_probe;
-  d.ckmag = (const uint16_t*)b;
-  b += sz_ck;
-  d.cnt = (const uint8_t*)b;
-  b += sz_cnt;
-  h->d_desc = (HandleDesc*)b;
-  b += sz_desc;
-  unsigned int* prep_status = (unsigned int*)b;
+    return s;
+  };
+  if ((st = h->tables.alloc(sz_tables)) != EFFORT_OK) return fail(st);
+  if ((st = tmp.alloc(sz_tmp)) != EFFORT_OK) return fail(st);
+  char* tb = (char*)h->tables.p;
+  d.lst = (const uint4*)tb;
+  d.wdense = (const uint16_t*)(tb + sz_lst);
+  d.probes = (const uint16_t*)(tb + sz_lst + sz_dense);
+  unsigned* ctl = (unsigned*)(tb + sz_lst + sz_dense + sz_probe);  // [0] chunk counter, [1] status
+  uint16_t* tvals = (uint16_t*)tmp.p;
+  uint8_t* tgaps = (uint8_t*)(tvals + (size_t)cap_chunks * kCS);
+  uint16_t* thead = (uint16_t*)(tgaps + (size_t)cap_chunks * kCS);
 
   cudaStream_t s = (cudaStream_t)stream;
   h->last_stream = s;
-  cudaError_t e = cudaMemsetAsync(h->storage, 0, total, s);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(h->d_desc, &d, sizeof(HandleDesc), cudaMemcpyHostToDevice, s);
+  cudaError_t e = cudaMemsetAsync(h->tables.p, 0, sz_tables, s);
   if (e == cudaSuccess)
-    e = launch_prep((const uint16_t*)W, h->d_desc, I, g.O, (uint16_t*)d.vals, (uint8_t*)d.idx, (uint16_t*)d.wdense,
-                    (uint16_t*)d.probes, (uint16_t*)d.ckmag, (uint8_t*)d.cnt, prep_status, s);
-  unsigned int status_h = 0;
-  if (e == cudaSuccess) e = cudaMemcpyAsync(&status_h, prep_status, 4, cudaMemcpyDeviceToHost, s);
+    e = launch_prep((const uint16_t*)W, I, O, n, P, dstride, prank, (uint16_t*)d.wdense, (uint16_t*)d.probes, tvals,
+                    tgaps, thead, (uint4*)d.lst, ctl, (unsigned)cap_chunks, ctl + 1, s);
+  unsigned ctl_h[2] = {0, 0};
+  if (e == cudaSuccess) e = cudaMemcpyAsync(ctl_h, ctl, 8, cudaMemcpyDeviceToHost, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
-  if (e != cudaSuccess) {
-    cudaGetLastError();
-    cudaFree(h->storage);
-    delete h;
-    return EFFORT_ERR_CUDA;
-  }
-  if (status_h & kStatusNonfiniteW) {
-    cudaFree(h->storage);
-    delete h;
-    return EFFORT_ERR_NONFINITE;
-  }
-  st = alloc_ws(g, 1, &h->ws, &h->slot);
-  if (st != EFFORT_OK) {
-    cudaFree(h->storage);
-    delete h;
-    return st;
-  }
-  if (cudaMalloc(&h->stage, stage_out_offset(g.I) + (size_t)g.O * 4) != cudaSuccess) {
-    cudaGetLastError();
-    cudaFree(h->ws.base);
-    cudaFree(h->storage);
-    delete h;
-    return EFFORT_ERR_NOMEM;
-  }
-  *out_handle = h;
-  return EFFORT_OK;
-}
+  if (e != cudaSuccess) return fail(EFFORT_ERR_CUDA);
+  if (ctl_h[1] & kStatusNonfiniteW) return fail(EFFORT_ERR_NONFINITE);
+  if (ctl_h[1] & kStatusInternal) return fail(EFFORT_ERR_DEVICE);
 
-static effort_status_t fill_job(effort_handle_t h, const WsPtrs& ws, const void* v, effort_dtype_t v_dtype,
-                                float effort, float* out, float* cutoff_out, uint64_t* count_out,
-                                uint32_t* rowlen_out, Job* j) {
-  if (!v || !out) return EFFORT_ERR_ARG;
-  if (v_dtype != EFFORT_F32 && v_dtype != EFFORT_F16) return EFFORT_ERR_ARG;
-  if (!effort_ok(effort)) return EFFORT_ERR_ARG;
-  const long long N = (long long)h->g.I * (long long)h->g.O;
-  const unsigned long long K = target_count(effort, N);
-  j->hd = h->hd;
-  j->v = v;
-  j->out = out;
-  j->cutoff_out = cutoff_out;
-  j->count_out = (unsigned long long*)count_out;
-  j->rowlen_out = rowlen_out;
-  j->ws = ws;
-  j->K = K;
-  j->mode = (K >= h->hd.kept_total) ? kModeAll : (K == 0 ? kModeNone : kModeSelect);
-  j->vdtype = (int)v_dtype;
-  j->dense_q16 = h->g.dense_q16;
+  // the used chunks into storage of the exact size
+  const size_t nch = ctl_h[0];
+  d.total_chunks = (unsigned)nch;
+  const size_t cv = align_up(nch * kCS * 2, 256), cg = align_up(nch * kCS, 256), chd = align_up(nch * 2 + 2, 256);
+  if ((st = h->chunks.alloc(cv + cg + chd)) != EFFORT_OK) return fail(st);
+  char* cb = (char*)h->chunks.p;
+  d.vals = (const uint16_t*)cb;
+  d.gaps = (const uint8_t*)(cb + cv);
+  d.head = (const uint16_t*)(cb + cv + cg);
+  e = cudaMemcpyAsync((void*)d.vals, tvals, nch * kCS * 2, cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync((void*)d.gaps, tgaps, nch * kCS, cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync((void*)d.head, thead, nch * 2, cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return fail(EFFORT_ERR_CUDA);
+  tmp.release();
+  h->storage_bytes = h->chunks.bytes + h->tables.bytes;
+
+  // per-call scratch and the host-call staging buffer
+  if ((st = h->ws.alloc(scratch_bytes(h->g))) != EFFORT_OK) return fail(st);
+  h->slot = carve((char*)h->ws.p, h->g);
+  if (clear_scratch(h->slot, s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess) return fail(EFFORT_ERR_CUDA);
+  if ((st = h->stage.alloc(stage_out_offset(I) + (size_t)O * 4)) != EFFORT_OK) return fail(st);
+  *out_handle = h;
   return EFFORT_OK;
 }
 
 effort_status_t effort_gemv_ex(effort_handle_t h, const void* v, effort_dtype_t v_dtype, float effort, float* out,
                                float* cutoff_out, uint64_t* count_out, uint32_t* rowlen_out, void* stream) {
   if (!h) return EFFORT_ERR_ARG;
-  Jobs<1> jobs;
-  effort_status_t st = fill_job(h, h->slot, v, v_dtype, effort, out, cutoff_out, count_out, rowlen_out, &jobs.j[0]);
+  Job job;
+  effort_status_t st = fill_job(h, h->slot, v, v_dtype, effort, out, cutoff_out, count_out, rowlen_out, &job);
   if (st != EFFORT_OK) return st;
   DeviceGuard guard(h->dev);
   cudaStream_t s = (cudaStream_t)stream;
   h->last_stream = s;
-  cudaError_t e = launch_cutoff(jobs, h->g.I, h->g.cl, s);
-  if (e == cudaSuccess) e = launch_mac(jobs, h->g.T, h->g.S, s);
-  if (e != cudaSuccess) {
+  if (launch_effort(job, h->g.nb, h->g.smem, s) != cudaSuccess) {
     cudaGetLastError();
     return EFFORT_ERR_CUDA;
   }
   return EFFORT_OK;
 }
 
-effort_status_t effort_gemv_split(effort_handle_t h, const void* v, effort_dtype_t v_dtype, float effort, float* out,
-                                  float* cutoff_out, uint64_t* count_out, void* mid_event, void* stream) {
-  if (!h || !mid_event) return EFFORT_ERR_ARG;
-  Jobs<1> jobs;
-  effort_status_t st = fill_job(h, h->slot, v, v_dtype, effort, out, cutoff_out, count_out, nullptr, &jobs.j[0]);
+effort_status_t effort_gemv_timed(effort_handle_t h, const void* v, effort_dtype_t v_dtype, float effort, float* out,
+                                  uint64_t* marks, void* stream) {
+  if (!h || !marks) return EFFORT_ERR_ARG;
+  Job job;
+  effort_status_t st = fill_job(h, h->slot, v, v_dtype, effort, out, nullptr, nullptr, nullptr, &job);
   if (st != EFFORT_OK) return st;
+  job.marks = (unsigned long long*)marks;
   DeviceGuard guard(h->dev);
   cudaStream_t s = (cudaStream_t)stream;
   h->last_stream = s;
-  cudaError_t e = launch_cutoff(jobs, h->g.I, h->g.cl, s);
-  // under stream capture the event is recorded as an external event-record
-  // node, so that the phases of a captured graph can be timed too
-  if (e == cudaSuccess) {
-    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
-    e = cudaStreamIsCapturing(s, &cap);
-    if (e == cudaSuccess)
-      e = (cap == cudaStreamCaptureStatusActive)
-              ? cudaEventRecordWithFlags((cudaEvent_t)mid_event, s, cudaEventRecordExternal)
-              : cudaEventRecord((cudaEvent_t)mid_event, s);
-  }
-  if (e == cudaSuccess) e = launch_mac(jobs, h->g.T, h->g.S, s);
-  if (e != cudaSuccess) {
+  if (launch_effort(job, h->g.nb, h->g.smem, s) != cudaSuccess) {
     cudaGetLastError();
     return EFFORT_ERR_CUDA;
   }
+  return EFFORT_OK;
+}
+
+effort_status_t effort_grid_blocks(effort_handle_t h, int32_t* blocks) {
+  if (!h || !blocks) return EFFORT_ERR_ARG;
+  *blocks = h->g.nb;
   return EFFORT_OK;
 }
 
@@ -411,14 +433,13 @@ effort_status_t effort_gemv_host(effort_handle_t h, const void* v_host, effort_d
   if (!effort_ok(effort)) return EFFORT_ERR_ARG;
   DeviceGuard guard(h->dev);
   cudaStream_t s = (cudaStream_t)stream;
-  // page-locked memory mapped into the device's address space is read and
-  // written in place by the kernels; other host memory goes through the
-  // staging buffer with one copy each way
+  // page-locked v mapped into the device's address space is read in place by
+  // the kernel; other host memory is copied into the staging buffer.  out is
+  // accumulated with device-memory reductions, so it always goes through the
+  // staging buffer and one copy back
   void* mv = mapped_host_pointer(v_host);
-  void* mo = mapped_host_pointer(out_host);
-  void* d_v = mv ? mv : h->stage;
-  float* d_out = mo ? static_cast<float*>(mo)
-                    : reinterpret_cast<float*>(static_cast<char*>(h->stage) + stage_out_offset(h->g.I));
+  void* d_v = mv ? mv : h->stage.p;
+  float* d_out = reinterpret_cast<float*>(static_cast<char*>(h->stage.p) + stage_out_offset(h->g.I));
   const size_t vbytes = (size_t)h->g.I * (v_dtype == EFFORT_F16 ? 2 : 4);
   if (!mv && cudaMemcpyAsync(d_v, v_host, vbytes, cudaMemcpyHostToDevice, s) != cudaSuccess) {
     cudaGetLastError();
@@ -426,7 +447,7 @@ effort_status_t effort_gemv_host(effort_handle_t h, const void* v_host, effort_d
   }
   const effort_status_t st = effort_gemv_ex(h, d_v, v_dtype, effort, d_out, nullptr, nullptr, nullptr, stream);
   if (st != EFFORT_OK) return st;
-  if (!mo && cudaMemcpyAsync(out_host, d_out, (size_t)h->g.O * 4, cudaMemcpyDeviceToHost, s) != cudaSuccess) {
+  if (cudaMemcpyAsync(out_host, d_out, (size_t)h->g.O * 4, cudaMemcpyDeviceToHost, s) != cudaSuccess) {
     cudaGetLastError();
     return EFFORT_ERR_CUDA;
   }
@@ -442,10 +463,15 @@ effort_status_t effort_check(effort_handle_t h) {
   DeviceGuard guard(h->dev);
   unsigned int st = 0;
   if (cudaStreamSynchronize(h->last_stream) != cudaSuccess) return EFFORT_ERR_CUDA;
-  if (cudaMemcpy(&st, h->slot.status, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return EFFORT_ERR_CUDA;
-  if (st && cudaMemset(h->slot.status, 0, 4) != cudaSuccess) return EFFORT_ERR_CUDA;
+  if (cudaMemcpy(&st, h->slot.hdr + kHdrStatus, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return EFFORT_ERR_CUDA;
+  if (st) {
+    // a timed-out grid leaves the barrier counter and histograms mid-call:
+    // start the scratch over (the status word with it)
+    if (clear_scratch(h->slot, h->last_stream) != cudaSuccess || cudaStreamSynchronize(h->last_stream) != cudaSuccess)
+      return EFFORT_ERR_CUDA;
+  }
+  if (st & (kStatusInternal | kStatusTimeout)) return EFFORT_ERR_DEVICE;
   if (st & kStatusNonfiniteV) return EFFORT_ERR_NONFINITE;
-  if (st & kStatusInternal) return EFFORT_ERR_DEVICE;
   return EFFORT_OK;
 }
 
@@ -456,20 +482,24 @@ effort_status_t effort_workspace_create(int64_t in_dim, int64_t out_dim, int32_t
   if (out_dim > EFFORT_MAX_OUT_DIM || in_dim > EFFORT_MAX_IN_DIM) return EFFORT_ERR_UNSUPPORTED;
   effort_workspace_s* w = new (std::nothrow) effort_workspace_s();
   if (!w) return EFFORT_ERR_NOMEM;
-  cudaGetDevice(&w->dev);
-  effort_status_t st = make_geometry(in_dim, out_dim, &w->g);
-  if (st != EFFORT_OK) {
+  if (cudaGetDevice(&w->dev) != cudaSuccess) {
+    cudaGetLastError();
     delete w;
-    return st;
+    return EFFORT_ERR_CUDA;
   }
-  w->slots = new (std::nothrow) WsPtrs[max_pairs];
-  if (!w->slots) {
-    delete w;
-    return EFFORT_ERR_NOMEM;
+  effort_status_t st = make_geometry(in_dim, out_dim, (int)out_dim, &w->g);
+  if (st == EFFORT_OK) st = w->ws.alloc(scratch_bytes(w->g));
+  if (st == EFFORT_OK) {
+    w->slot = carve((char*)w->ws.p, w->g);
+    if (clear_scratch(w->slot, nullptr) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) st = EFFORT_ERR_CUDA;
   }
-  st = alloc_ws(w->g, max_pairs, &w->ws, w->slots);
+  const size_t dense_bytes = align_up((size_t)w->g.S_dense * w->g.T * 256 * 4, 256) + align_up((size_t)w->g.T * 4, 256);
+  if (st == EFFORT_OK) st = w->dense_part.alloc(dense_bytes);
+  if (st == EFFORT_OK && cudaMemset(w->dense_part.p, 0, dense_bytes) != cudaSuccess) st = EFFORT_ERR_CUDA;
   if (st != EFFORT_OK) {
-    delete[] w->slots;
+    cudaGetLastError();
+    w->ws.release();
+    w->dense_part.release();
     delete w;
     return st;
   }
@@ -483,9 +513,9 @@ effort_status_t effort_workspace_destroy(effort_workspace_t w) {
   {
     DeviceGuard guard(w->dev);
     cudaStreamSynchronize(w->last_stream);
-    cudaFree(w->ws.base);
+    w->ws.release();
+    w->dense_part.release();
   }
-  delete[] w->slots;
   delete w;
   return EFFORT_OK;
 }
@@ -501,26 +531,22 @@ effort_status_t effort_gemv_batched(effort_workspace_t ws, const effort_handle_t
   const size_t vsz = (v_dtype == EFFORT_F16) ? 2 : 4;
   for (int p = 0; p < n_pairs; ++p) {
     if (hidx[p] < 0 || vidx[p] < 0) return EFFORT_ERR_ARG;
+    effort_handle_t h = handles[hidx[p]];
+    if (!h || h->g.I != I || h->g.O != O || !effort_ok(efforts[p])) return EFFORT_ERR_ARG;
   }
   DeviceGuard guard(ws->dev);
   cudaStream_t s = (cudaStream_t)stream;
   ws->last_stream = s;
-  for (int p0 = 0; p0 < n_pairs; p0 += kMaxJobs) {
-    const int nj = (n_pairs - p0 < kMaxJobs) ? n_pairs - p0 : kMaxJobs;
-    Jobs<kMaxJobs> jobs;
-    memset(&jobs, 0, sizeof(jobs));
-    for (int q = 0; q < nj; ++q) {
-      const int p = p0 + q;
-      effort_handle_t h = handles[hidx[p]];
-      if (!h || h->g.I != I || h->g.O != O) return EFFORT_ERR_ARG;
-      effort_status_t st = fill_job(h, ws->slots[p], (const char*)V + (size_t)vidx[p] * I * vsz, v_dtype, efforts[p],
-                                    OUT + (size_t)p * O, cutoffs_out ? cutoffs_out + p : nullptr,
-                                    counts_out ? counts_out + p : nullptr, nullptr, &jobs.j[q]);
-      if (st != EFFORT_OK) return st;
-    }
-    cudaError_t e = launch_cutoff_batch(jobs, nj, I, ws->g.cl, s);
-    if (e == cudaSuccess) e = launch_mac_batch(jobs, nj, ws->g.T, ws->g.S, s);
-    if (e != cudaSuccess) {
+  // one grid per pair, all on one stream: each grid waits for the one before
+  // it, so the pairs share the workspace's scratch
+  for (int p = 0; p < n_pairs; ++p) {
+    effort_handle_t h = handles[hidx[p]];
+    Job job;
+    effort_status_t st = fill_job(h, ws->slot, (const char*)V + (size_t)vidx[p] * I * vsz, v_dtype, efforts[p],
+                                  OUT + (size_t)p * O, cutoffs_out ? cutoffs_out + p : nullptr,
+                                  counts_out ? counts_out + p : nullptr, nullptr, &job);
+    if (st != EFFORT_OK) return st;
+    if (launch_effort(job, ws->g.nb, ws->g.smem, s) != cudaSuccess) {
       cudaGetLastError();
       return EFFORT_ERR_CUDA;
     }
@@ -537,8 +563,10 @@ effort_status_t effort_dense_gemv(effort_workspace_t ws, const void* W, int64_t 
   DeviceGuard guard(ws->dev);
   cudaStream_t s = (cudaStream_t)stream;
   ws->last_stream = s;
-  cudaError_t e = launch_dense((const uint16_t*)W, ws->g.I, ws->g.O, v, (int)v_dtype, out, ws->slots[0].part,
-                               ws->slots[0].tilecnt, ws->g.T, ws->g.S_dense, s);
+  float* part = (float*)ws->dense_part.p;
+  unsigned* tilecnt = (unsigned*)((char*)ws->dense_part.p + align_up((size_t)ws->g.S_dense * ws->g.T * 256 * 4, 256));
+  cudaError_t e = launch_dense((const uint16_t*)W, ws->g.I, ws->g.O, v, (int)v_dtype, out, part, tilecnt, ws->g.T,
+                               ws->g.S_dense, s);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return EFFORT_ERR_CUDA;
@@ -552,7 +580,7 @@ effort_status_t effort_get_info(effort_handle_t h, int64_t* in_dim, int64_t* out
   if (in_dim) *in_dim = h->g.I;
   if (out_dim) *out_dim = h->g.O;
   if (keep_fraction) *keep_fraction = h->keep;
-  if (device_bytes) *device_bytes = h->storage_bytes + h->ws.bytes;
+  if (device_bytes) *device_bytes = h->storage_bytes;
   return EFFORT_OK;
 }
 
@@ -561,20 +589,21 @@ effort_status_t effort_get_layout(effort_handle_t h, effort_layout_t* L) {
   L->in_dim = h->g.I;
   L->out_dim = h->g.O;
   L->n_kept = h->hd.n;
-  L->n_tiles = h->hd.T;
-  L->bucket_cap = kCap;
-  L->ck_step = h->hd.H;
-  L->n_ck = h->hd.C;
+  L->n_panels = h->hd.P;
+  L->panel_width = kPW;
+  L->chunk_slots = kCS;
+  L->store_num = kStoreNum;
+  L->store_den = kStoreDen;
   L->n_probes = kP;
+  L->dense_stride = h->hd.dstride;
+  L->total_chunks = h->hd.total_chunks;
   L->vals = h->hd.vals;
-  L->idx = h->hd.idx;
-  L->probes = h->hd.probes;
-  L->ckmag = h->hd.ckmag;
-  L->cnt = h->hd.cnt;
+  L->gaps = h->hd.gaps;
+  L->head = h->hd.head;
+  L->lists = h->hd.lst;
   L->wdense = h->hd.wdense;
-  L->rec = h->slot.rec;
-  L->gcnt = h->slot.gcnt;
-  L->n_groups = h->g.G;
+  L->probes = h->hd.probes;
+  L->scratch_bytes = h->ws.bytes;
   return EFFORT_OK;
 }
 
@@ -583,37 +612,33 @@ effort_status_t effort_destroy(effort_handle_t h) {
   {
     DeviceGuard guard(h->dev);
     cudaStreamSynchronize(h->last_stream);
-    cudaFree(h->stage);
-    cudaFree(h->ws.base);
-    cudaFree(h->storage);
+    h->stage.release();
+    h->ws.release();
+    h->chunks.release();
+    h->tables.release();
   }
   delete h;
   return EFFORT_OK;
 }
 
-}  // extern "C"
-
-namespace effort {
-
-// For entry points that bring their own per-call scratch: the handle's device
-// and the launch geometry of one call.
-effort_status_t handle_call_geometry(effort_handle_t h, int* dev, int* I, int* T, int* G, int* S, int* cl) {
-  if (!h) return EFFORT_ERR_ARG;
-  *dev = h->dev;
-  *I = h->g.I;
-  *T = h->g.T;
-  *G = h->g.G;
-  *S = h->g.S;
-  *cl = h->g.cl;
+effort_status_t effort_last_call_bytes(effort_handle_t h, uint64_t* dense_bytes, uint64_t* sparse_bytes) {
+  if (!h || !dense_bytes || !sparse_bytes) return EFFORT_ERR_ARG;
+  DeviceGuard guard(h->dev);
+  unsigned long long b[2] = {0, 0};
+  if (cudaStreamSynchronize(h->last_stream) != cudaSuccess ||
+      cudaMemcpy(b, h->slot.hdr + kHdrBytesLast, 16, cudaMemcpyDeviceToHost) != cudaSuccess) {
+    cudaGetLastError();
+    return EFFORT_ERR_CUDA;
+  }
+  *dense_bytes = b[0];
+  *sparse_bytes = b[1];
   return EFFORT_OK;
 }
 
-// The same argument checks and job description as effort_gemv_ex, with the
-// caller's scratch in place of the handle's.
-effort_status_t handle_fill_job(effort_handle_t h, const WsPtrs& ws, const void* v, effort_dtype_t v_dtype,
-                                float effort, float* out, float* cutoff_out, uint64_t* count_out, Job* j) {
-  if (!h) return EFFORT_ERR_ARG;
-  return fill_job(h, ws, v, v_dtype, effort, out, cutoff_out, count_out, nullptr, j);
+effort_status_t effort_device_bytes_held(uint64_t* bytes) {
+  if (!bytes) return EFFORT_ERR_ARG;
+  *bytes = g_live_bytes.load();
+  return EFFORT_OK;
 }
 
-}  // namespace effort
+}  // extern "C"

@@ -10,6 +10,8 @@
 
 namespace effort {
 
+constexpr int kTW = 256;  // columns of one output tile
+
 template <typename VT>
 __global__ void __launch_bounds__(kDenseThreads, 4) k_dense_gemv(const uint16_t* __restrict__ W, int I, int O,
                                                               const VT* __restrict__ v, float* out, float* part,

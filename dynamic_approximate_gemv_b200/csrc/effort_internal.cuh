@@ -1,20 +1,29 @@
 // Internal definitions shared by the library's kernels and host code.
 //
-// Storage of a prepared matrix W [I x O] (binary16), per row i with kept count
-// n = floor(keep * O + 1/2):
-//   * buckets: tile t covers columns [256 t, 256 t + 256).  Bucket (i, t) holds
-//     the kept entries of row i in tile t, ordered by |w| descending (ties:
-//     lower column first), as fp16 value bits + u8 local column, at entry
-//     offset (t * I + i) * kCap.  Unused slots are +0.0 / 0.
-//   * wdense: [I][T * 256] fp16, kept weights at their columns, 0 elsewhere.
+// Storage of a prepared matrix W [I x O] (binary16).  Row i's order is |w|
+// descending with ties to the lower column, and its first n = floor(keep * O
+// + 1/2) entries are kept.  The columns are cut into panels of kPW (2048)
+// columns; panel p holds columns [kPW p, kPW p + kPW).
+//   * lists: for every (row i, panel p), the kept entries of row i whose
+//     column lies in panel p, in row i's order.  Only the leading
+//     ceil(n_ip * kStoreNum / kStoreDen) of them are stored (n_ip = the list's
+//     kept entries); a call that needs more of a list reads the row from the
+//     dense copy instead.  The stored part is cut into chunks of kCS slots.
+//     A chunk holds a run of consecutive ranks, sorted by column, as binary16
+//     value bits (vals) and 8-bit column gaps (gaps): the first gap counts
+//     from column -1 of the panel, every further one from the previous slot.
+//     A gap of more than 255 is bridged by filler slots (value +0, gap 255);
+//     the chunk is padded to kCS slots with (value +0, gap 0).  Fillers and
+//     pads have magnitude 0, so no call with a positive cutoff uses them, and
+//     at cutoff 0 they add +0 to a column of the panel.
+//   * head: per chunk, the magnitude bits of its first (largest) rank.
+//   * lst:  per (i, p) {first chunk, stored chunks, tail, n_ip}, where tail
+//     is the magnitude bits of the first rank that is not stored (0 when the
+//     whole list is stored) and n_ip the list's kept entries.
+//   * wdense: [I][dstride] fp16, kept weights at their columns, +0 elsewhere
+//     (dstride = O rounded up to a multiple of 256).
 //   * probes: [I][16] |w| bits at the midpoint ranks of 16 equal segments of
 //     the kept list (the `get_probes` step of the pages' pseudo-code).
-//   * ckmag: [I][C + 1]: rank-0 magnitude, then the magnitude at the last rank
-//     of each checkpoint block of H ranks (block k ends at min((k+1)H, n)).
-//   * cnt: [I][C][T] u8: entries of tile t among the ranks before the end of
-//     checkpoint block k, saturated at 255.
-// Per call (one "job"): a cutoff c, per-row dispatch records grouped by 32
-// rows, and split-K partial sums of each output tile.
 #pragma once
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -22,63 +31,65 @@
 
 namespace effort {
 
-constexpr int kTW = 256;         // output-tile width (u8 local column)
-constexpr int kCap = 256;        // bucket capacity (entries)
-constexpr int kP = 16;           // probes per row
-constexpr int kCutThreads = 1024;
-#ifndef EFFORT_MAC_THREADS
-#define EFFORT_MAC_THREADS 384  // multiply kernel block size
-#endif
-#ifndef EFFORT_MAC_BLOCKS_PER_SM
-#define EFFORT_MAC_BLOCKS_PER_SM 2  // resident multiply blocks per SM the register budget is sized for
-#endif
-constexpr int kMacThreads = EFFORT_MAC_THREADS;
-constexpr int kMacBlocksPerSM = EFFORT_MAC_BLOCKS_PER_SM;
-constexpr int kMacWarps = kMacThreads / 32;
+constexpr int kP = 16;            // probes per row
+constexpr int kPW = 2048;         // panel width (columns)
+constexpr int kStripe = 256;      // dense stripe: 32 lanes x 8 columns
+constexpr int kCS = 64;           // slots per chunk: 8 lanes x 8 slots
+constexpr int kLanesPerChunk = kCS / 8;
+constexpr int kStoreNum = 3, kStoreDen = 8;  // stored share of every list
+constexpr int kThreads = 1024;    // threads of the matvec kernel (one block per SM)
+constexpr int kWarps = kThreads / 32;
 constexpr int kPrepThreads = 1024;
 constexpr int kDenseThreads = 256;
-constexpr int kMaxJobs = 16;     // pairs per launch
-constexpr int kGroupRows = 32;   // dispatch records are grouped by 32 rows
-constexpr int kRecPerGroup = 32; // one 8-byte record per row of a group
+constexpr int kDenseRowsPerItem = 8;  // dense rows a warp accumulates per stripe item
+constexpr int kMaxPanels = 16;        // 32768 / 2048
 
 // call modes decided on the host from K and the kept count
 enum : int { kModeSelect = 0, kModeAll = 1, kModeNone = 2 };
 // device status bits
-enum : unsigned { kStatusNonfiniteV = 1u, kStatusNonfiniteW = 2u, kStatusInternal = 4u };
-// dispatch classes
-enum : int { kClassOff = 0, kClassSparse = 1, kClassDense = 2 };
+enum : unsigned { kStatusNonfiniteV = 1u, kStatusNonfiniteW = 2u, kStatusInternal = 4u, kStatusTimeout = 8u };
 
-// Device-resident description of a prepared matrix (written once at prepare).
+// radix-select digits of the non-negative fp32 chart: bits [30:19], [18:9], [8:0]
+constexpr int kBins0 = 4096, kBins1 = 1024, kBins2 = 512;
+constexpr int kCandCap = 4096;     // crossing-bin candidates resolved in one block
+
+// Device-resident description of a prepared matrix (passed by value).
 struct HandleDesc {
-  const uint16_t* vals;
-  const uint8_t* idx;
-  const uint16_t* wdense;
-  const uint16_t* probes;
-  const uint16_t* ckmag;
-  const uint8_t* cnt;
-  int I, O, T, n, C, H, dstride;
-  int pad0;
+  const uint16_t* vals;    // [total chunks * kCS]
+  const uint8_t* gaps;     // [total chunks * kCS]
+  const uint16_t* head;    // [total chunks]
+  const uint4* lst;        // [I][P]
+  const uint16_t* wdense;  // [I][dstride]
+  const uint16_t* probes;  // [I][kP]
+  int I, O, n, P, dstride;
+  unsigned total_chunks;
   unsigned long long kept_total;
-  int prank[kP];  // probe ranks (-1 for empty segments)
-  int pw[kP];     // probe weights (entries each probe stands for)
+  int pw[kP];              // probe weights (entries each probe stands for)
 };
 
-// Per-job scratch.
+// Per-call scratch in device memory.  The header words and the first-digit
+// histogram must be zero before a call (the library clears them at
+// allocation and every call leaves them zero, except after a timeout).
 struct WsPtrs {
-  float* c;                     // the cutoff
-  unsigned long long* count;    // running |S|
-  unsigned int* done;           // CTAs of the multiply kernel that finished
-  unsigned int* tilecnt;        // [T] split-K arrivals per tile
-  uint2* rec;                   // [G][32] dispatch records {v bits, tau (fp16 bits) | row << 16}:
-                                //   sparse rows at [0, ns), dense rows at [ns, ns + nd)
-  unsigned int* gcnt;           // [G] ns | nd << 8
-  unsigned char* ut;            // [G][T][32]: read bound U of sparse slot p of group g in tile t
-  float* part;                  // per-tile partial sums of the CTAs that share a tile
-  unsigned int* status;         // sticky device status bits
+  unsigned* hdr;              // see kHdr* below
+  unsigned long long* bar;    // grid-barrier counter (monotonic)
+  unsigned long long* count;  // running |S|
+  unsigned* ghist0;           // [kBins0]
+  unsigned* ghist1;           // [kBins1]
+  unsigned* ghist2;           // [kBins2]
+  uint2* cand;                // [kCandCap] {chart bits, weight}
+  unsigned* info;             // [I][P]: bit 31 dense, bits 0..30 chunks to read
+  unsigned* rowpre;           // [I][P]: work bytes of the owner block's rows before row i
+  unsigned* ctot;             // [nb][P]: work bytes of each owner block's rows
 };
+// header words: status, candidate count, then 64-bit byte counters: the dense
+// and sparse bytes the running call plans to read (words 8..11) and those of
+// the last finished call (words 12..15)
+enum : int { kHdrStatus = 0, kHdrCand = 1, kHdrDone = 2, kHdrBytesRun = 8, kHdrBytesLast = 12, kHdrWords = 64 };
 
 struct Job {
-  HandleDesc hd;  // by value: kernels read it from the parameter bank
+  HandleDesc hd;
+  unsigned barrier_nb;  // blocks each grid-wide barrier waits for (the grid size)
   const void* v;
   float* out;
   float* cutoff_out;
@@ -87,38 +98,31 @@ struct Job {
   WsPtrs ws;
   unsigned long long K;
   int mode;
-  int vdtype;     // 0 f32, 1 f16
-  int dense_q16;  // a row is read densely once this share (x 65536) of it is surely used
-  int pad0;
+  int vdtype;  // 0 f32, 1 f16
+  unsigned long long* marks;  // nullable: [grid][kMarks] phase times (measurement entry point)
 };
+constexpr int kMarks = 16;
 
-template <int NJ>
-struct Jobs {
-  Job j[NJ];
-};
+// Rows of the chart each block of an nb-block grid owns during the cutoff.
+__host__ __device__ inline int rows_per_block(int I, int nb) { return (I + nb - 1) / nb; }
 
-// Cutoff cluster geometry: rows per CTA rounded to whole 32-row groups.
-__host__ __device__ inline int cut_rows_per_cta(int I, int cl) {
-  int rp = (I + cl - 1) / cl;
-  return (rp + kGroupRows - 1) / kGroupRows * kGroupRows;
-}
-// radix-select digits: bits [30:19], [18:9], [8:0] of the non-negative fp32 chart
-constexpr int kBins0 = 4096, kBins1 = 1024, kBins2 = 512;
-constexpr int kCandLocal = 2048;  // crossing-bin candidates one cutoff CTA can hold
-constexpr int kCandTotal = 4096;  // candidates gathered from the whole cluster
-// dynamic shared memory of a cutoff CTA: chart, v, the first-pass histogram,
-// its candidate list, and one area shared by the merged histogram, the
-// gathered candidates and the fallback passes
-__host__ __device__ inline size_t cut_union_bytes() {
-  const size_t merged = (size_t)kBins0 * 4;
-  const size_t gathered = (size_t)kCandTotal * 6;
-  const size_t fallback = 2 * (size_t)(kBins1 + kBins2) * 4;
-  size_t m = merged > gathered ? merged : gathered;
-  return m > fallback ? m : fallback;
-}
-__host__ __device__ inline size_t cut_smem_bytes(int I, int cl) {
-  const size_t rp = (size_t)cut_rows_per_cta(I, cl);
-  return rp * kP * 4 + rp * 4 + (size_t)kBins0 * 4 + (size_t)kCandLocal * 6 + cut_union_bytes() + 64;
+// Dynamic shared memory of the matvec kernel.
+__host__ __device__ inline size_t smem_layout(int I, int nb, size_t* off_chart, size_t* off_hist, size_t* off_cand,
+                                              size_t* off_lists, size_t* off_ctl) {
+  const size_t rp = (size_t)rows_per_block(I, nb);
+  size_t o = (size_t)kPW * 4;                         // panel accumulator
+  *off_chart = o;
+  o += rp * kP * 4 + rp * 4 + 64;                     // chart bits and |v| of the owned rows
+  o = (o + 15) / 16 * 16;
+  *off_hist = o;
+  o += (size_t)kBins0 * 4;                            // first-digit histogram / later digits
+  *off_cand = o;
+  o += (size_t)kCandCap * 8;                          // gathered candidates
+  *off_lists = o;
+  o += 64 * 1024;                                     // work lists of the block
+  *off_ctl = o;
+  o += (size_t)(128 + kMaxPanels * (nb + 1)) * 4;     // control words and prefix tables
+  return o;
 }
 
 }  // namespace effort

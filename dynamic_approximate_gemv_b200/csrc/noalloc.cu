@@ -7,11 +7,13 @@
 // before the first call.
 //
 // The scratch is one static array per device (every module-scope __device__
-// variable exists once per device context).  Its address is taken once per
-// device with cudaGetSymbolAddress, with that device current, on the first
-// call that runs there.  Every call then clears the words that must start at
-// zero with one cudaMemsetAsync on the call's stream and launches the same
-// two kernels as effort_gemv_ex.
+// variable exists once per device context).  Its address is taken with
+// cudaGetSymbolAddress, with that device current, on the first call that runs
+// in a given context of that device, and taken again if the context changed
+// since (a cudaDeviceReset creates a new primary context, in which the module
+// and its array are loaded anew).  Every call then clears the words that must
+// start at zero with one cudaMemsetAsync on the call's stream and launches
+// the same kernel as effort_gemv_ex.
 //
 // All calls on one device share the array: calls that overlap on the GPU
 // (different streams without ordering, or concurrent host threads) race and
@@ -22,11 +24,13 @@
 #include "effort_internal.cuh"
 
 namespace effort {
-cudaError_t launch_cutoff(const Jobs<1>& jobs, int I, int cl, cudaStream_t stream);
-cudaError_t launch_mac(const Jobs<1>& jobs, int T, int S, cudaStream_t stream);
-effort_status_t handle_call_geometry(effort_handle_t h, int* dev, int* I, int* T, int* G, int* S, int* cl);
+size_t handle_scratch_bytes(effort_handle_t h);
+size_t handle_scratch_zero_bytes();
+WsPtrs handle_carve(effort_handle_t h, char* base);
+int handle_device(effort_handle_t h);
 effort_status_t handle_fill_job(effort_handle_t h, const WsPtrs& ws, const void* v, effort_dtype_t v_dtype,
                                 float effort, float* out, float* cutoff_out, uint64_t* count_out, Job* j);
+cudaError_t handle_launch(effort_handle_t h, const Job& j, cudaStream_t s);
 }  // namespace effort
 
 using namespace effort;
@@ -40,48 +44,43 @@ __device__ __align__(256) unsigned char g_static_scratch[kScratchBytes];
 
 std::mutex g_mu;
 void* g_scratch_ptr[kMaxDevices] = {};
+void* g_scratch_ctx[kMaxDevices] = {};
 
-inline size_t align256(size_t x) { return (x + 255) / 256 * 256; }
-
-// Bytes of scratch one call needs: header (c, count, done, status), the
-// per-tile arrival counters, the dispatch tables and the split-K partials.
-size_t scratch_bytes(int T, int G, int S) {
-  return 256 + align256((size_t)T * 4) + align256((size_t)G * 4) + align256((size_t)G * T * 32) +
-         align256((size_t)G * kRecPerGroup * 8) + align256((size_t)S * T * kTW * 4);
+// The calling thread's current context, through the driver entry point the
+// runtime hands out (no link-time dependency on the driver library).
+typedef int (*CtxGetCurrentFn)(void**);
+void* current_context() {
+  static CtxGetCurrentFn fn = nullptr;
+  static bool looked = false;
+  if (!looked) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(f);
+    else
+      cudaGetLastError();
+    looked = true;
+  }
+  void* ctx = nullptr;
+  if (!fn || fn(&ctx) != 0) return nullptr;
+  return ctx;
 }
 
-// Carves the scratch in the same order as the handle's own workspace.
-WsPtrs carve(char* b, int T, int G) {
-  WsPtrs w;
-  w.c = (float*)(b + 0);
-  w.count = (unsigned long long*)(b + 8);
-  w.done = (unsigned int*)(b + 16);
-  w.status = (unsigned int*)(b + 20);
-  b += 256;
-  w.tilecnt = (unsigned int*)b;
-  b += align256((size_t)T * 4);
-  w.gcnt = (unsigned int*)b;
-  b += align256((size_t)G * 4);
-  w.ut = (unsigned char*)b;
-  b += align256((size_t)G * T * 32);
-  w.rec = (uint2*)b;
-  b += align256((size_t)G * kRecPerGroup * 8);
-  w.part = (float*)b;
-  return w;
-}
-
-// Address of this device's copy of the array; looked up once per device.
-// The caller has made `dev` current.
+// Address of this device's copy of the array, looked up once per device and
+// context.  The caller has made `dev` current.
 effort_status_t scratch_for_device(int dev, char** out) {
   if (dev < 0 || dev >= kMaxDevices) return EFFORT_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_scratch_ptr[dev]) {
+  void* ctx = current_context();
+  if (!g_scratch_ptr[dev] || ctx != g_scratch_ctx[dev] || ctx == nullptr) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) {
       cudaGetLastError();
       return EFFORT_ERR_CUDA;
     }
     g_scratch_ptr[dev] = p;
+    g_scratch_ctx[dev] = ctx;
   }
   *out = (char*)g_scratch_ptr[dev];
   return EFFORT_OK;
@@ -109,11 +108,12 @@ struct CurrentDevice {
 extern "C" effort_status_t effort_gemv_static(effort_handle_t h, const void* v, effort_dtype_t v_dtype,
                                               float effort, float* out, float* cutoff_out, uint64_t* count_out,
                                               uint32_t* status_out, void* stream) {
-  int dev = 0, I = 0, T = 0, G = 0, S = 0, cl = 0;
-  effort_status_t st = handle_call_geometry(h, &dev, &I, &T, &G, &S, &cl);
+  if (!h) return EFFORT_ERR_ARG;
+  Job probe;
+  effort_status_t st = handle_fill_job(h, WsPtrs{}, v, v_dtype, effort, out, cutoff_out, count_out, &probe);
   if (st != EFFORT_OK) return st;
-  const size_t need = scratch_bytes(T, G, S);
-  if (need > kScratchBytes) return EFFORT_ERR_UNSUPPORTED;
+  if (handle_scratch_bytes(h) > kScratchBytes) return EFFORT_ERR_UNSUPPORTED;
+  const int dev = handle_device(h);
   CurrentDevice guard(dev);
   if (!guard.ok) {
     cudaGetLastError();
@@ -122,17 +122,17 @@ extern "C" effort_status_t effort_gemv_static(effort_handle_t h, const void* v, 
   char* base = nullptr;
   st = scratch_for_device(dev, &base);
   if (st != EFFORT_OK) return st;
-  const WsPtrs ws = carve(base, T, G);
-  Jobs<1> jobs;
-  st = handle_fill_job(h, ws, v, v_dtype, effort, out, cutoff_out, count_out, &jobs.j[0]);
+  const WsPtrs ws = handle_carve(h, base);
+  Job job;
+  st = handle_fill_job(h, ws, v, v_dtype, effort, out, cutoff_out, count_out, &job);
   if (st != EFFORT_OK) return st;
   cudaStream_t s = (cudaStream_t)stream;
-  // header and per-tile counters start at zero; everything else is written
-  // before it is read within the call
-  cudaError_t e = cudaMemsetAsync(base, 0, 256 + align256((size_t)T * 4), s);
-  if (e == cudaSuccess) e = launch_cutoff(jobs, I, cl, s);
-  if (e == cudaSuccess) e = launch_mac(jobs, T, S, s);
-  if (e == cudaSuccess && status_out) e = cudaMemcpyAsync(status_out, ws.status, 4, cudaMemcpyDeviceToDevice, s);
+  // header, barrier counter and histograms start at zero; everything else is
+  // written before it is read within the call
+  cudaError_t e = cudaMemsetAsync(base, 0, handle_scratch_zero_bytes(), s);
+  if (e == cudaSuccess) e = handle_launch(h, job, s);
+  if (e == cudaSuccess && status_out)
+    e = cudaMemcpyAsync(status_out, ws.hdr + kHdrStatus, 4, cudaMemcpyDeviceToDevice, s);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return EFFORT_ERR_CUDA;

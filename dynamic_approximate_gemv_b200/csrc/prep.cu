@@ -6,21 +6,41 @@
 // One thread block per row:
 //   1. keys = (0x7FFF - |w| bits) << 16 | column: ascending order of the keys
 //      is |w| descending with ties broken by the lower column (the author's
-//      CSR reply: rows are stored from the largest absolute value down).
-//   2. bitonic sort of the keys in shared memory.
-//   3. the first n ranks are kept (the post text: the least important weights
-//      of a row can be left out of memory altogether).
-//   4. probes at the midpoint ranks of 16 equal segments; checkpoint
-//      magnitudes every H ranks; the dense copy of the kept weights.
-//   5. one warp per output tile walks the sorted row in rank order and
-//      appends the tile's entries to its bucket (stable, so each bucket is
-//      sorted the same way), recording the running count at every
-//      checkpoint.
+//      CSR reply: rows are stored from the largest absolute value down);
+//      bitonic sort in shared memory.
+//   2. the first n ranks are kept (the post text: the least important weights
+//      of a row can be left out of memory altogether); probes at the midpoint
+//      ranks of 16 equal segments; the dense copy of the kept weights.
+//   3. per output panel of 2048 columns, one warp takes the row's kept entries
+//      of that panel in rank order (the author's reply on the format: each
+//      row is split into parts and only the needed parts are read), keeps the
+//      leading 3/8 of them, and cuts those into chunks of 64 slots: a chunk is
+//      a run of consecutive ranks, stored sorted by column with 8-bit column
+//      gaps (filler slots bridge gaps above 255, pad slots fill the chunk).
+//      The greedy cut takes as many ranks as fit in 64 slots.  Chunks are
+//      placed through a global counter; the host then copies the used part
+//      into storage of the exact size.
 #include "effort_internal.cuh"
 
-#define EFFORT_PREP_SMEM_MAX (32768 * 4)  // keys of the widest supported row
+#define EFFORT_PREP_KEYS_MAX 32768
+#define EFFORT_PREP_LIST_MAX 800  // >= ceil(3 * 2048 / 8) + 1 entries of one panel list
 
 namespace effort {
+
+struct PrepArgs {
+  const uint16_t* W;
+  int I, O, n, P, dstride, Np;
+  uint16_t* wdense;
+  uint16_t* probes;
+  uint16_t* vals;        // capacity cap_chunks * kCS
+  uint8_t* gaps;         // capacity cap_chunks * kCS
+  uint16_t* head;        // capacity cap_chunks
+  uint4* lst;            // [I][P]
+  unsigned* chunk_count; // global chunk allocator
+  unsigned cap_chunks;
+  unsigned* status;
+  int prank[kP];         // probe ranks (-1 for empty segments)
+};
 
 __device__ __forceinline__ void bitonic_sort_u32(uint32_t* s, int Np) {
   for (int k = 2; k <= Np; k <<= 1) {
@@ -40,18 +60,71 @@ __device__ __forceinline__ void bitonic_sort_u32(uint32_t* s, int Np) {
   }
 }
 
-__global__ void __launch_bounds__(kPrepThreads, 1)
-    k_prep_rows(const uint16_t* __restrict__ W, const HandleDesc* __restrict__ hdp, int Np, uint16_t* vals,
-                uint8_t* idx, uint16_t* wdense, uint16_t* probes, uint16_t* ckmag, uint8_t* cnt,
-                unsigned int* status) {
-  extern __shared__ uint32_t keys[];  // Np entries
-  const int I = hdp->I, O = hdp->O, T = hdp->T, n = hdp->n, C = hdp->C, H = hdp->H;
-  const int dstride = hdp->dstride;
-  const int i = blockIdx.x;
-  const uint16_t* row = W + (size_t)i * O;
+// Ascending bitonic sort of 64 values held by a warp: element `lane` in a0,
+// element `lane + 32` in a1.
+__device__ __forceinline__ void warp_sort64(unsigned& a0, unsigned& a1) {
+  const int lane = threadIdx.x & 31;
+  for (int k = 2; k <= 64; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      if (j == 32) {
+        const unsigned lo = min(a0, a1), hi = max(a0, a1);
+        a0 = lo;
+        a1 = hi;
+      } else {
+        const unsigned b0 = __shfl_xor_sync(0xFFFFFFFFu, a0, j), b1 = __shfl_xor_sync(0xFFFFFFFFu, a1, j);
+        const bool lower = (lane & j) == 0;
+        const bool asc0 = (lane & k) == 0, asc1 = ((lane + 32) & k) == 0;
+        a0 = (lower == asc0) ? min(a0, b0) : max(a0, b0);
+        a1 = (lower == asc1) ? min(a1, b1) : max(a1, b1);
+      }
+    }
+  }
+}
 
+// For t <= 64 panel-local columns of a chunk (sorted ascending in s0/s1, the
+// positions >= t hold 0xFFFFFFFF), the per-position gap from the previous
+// column (from -1 for position 0) and the filler slots it needs.
+__device__ __forceinline__ void chunk_gaps(unsigned s0, unsigned s1, int t, int& g0, int& g1, int& f0, int& f1) {
+  const int lane = threadIdx.x & 31;
+  const unsigned up0 = __shfl_up_sync(0xFFFFFFFFu, s0, 1), up1 = __shfl_up_sync(0xFFFFFFFFu, s1, 1);
+  const unsigned last0 = __shfl_sync(0xFFFFFFFFu, s0, 31);
+  const int prev0 = (lane == 0) ? -1 : (int)up0;
+  const int prev1 = (lane == 0) ? (int)last0 : (int)up1;
+  g0 = (lane < t) ? (int)s0 - prev0 : 0;
+  g1 = (lane + 32 < t) ? (int)s1 - prev1 : 0;
+  f0 = (lane < t) ? (g0 - 1) / 255 : 0;
+  f1 = (lane + 32 < t) ? (g1 - 1) / 255 : 0;
+}
+
+__device__ __forceinline__ int warp_sum(int x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xFFFFFFFFu, x, o);
+  return x;
+}
+
+// Slots a chunk of the list entries [q, q + t) takes (entries plus fillers).
+__device__ __forceinline__ int chunk_slots(const uint32_t* list, int q, int t, int pbase) {
+  const int lane = threadIdx.x & 31;
+  unsigned s0 = (lane < t) ? (list[q + lane] & 0xFFFFu) - pbase : 0xFFFFFFFFu;
+  unsigned s1 = (lane + 32 < t) ? (list[q + lane + 32] & 0xFFFFu) - pbase : 0xFFFFFFFFu;
+  warp_sort64(s0, s1);
+  int g0, g1, f0, f1;
+  chunk_gaps(s0, s1, t, g0, g1, f0, f1);
+  return t + warp_sum(f0 + f1);
+}
+
+__global__ void __launch_bounds__(kPrepThreads, 1) k_prep_rows(const __grid_constant__ PrepArgs a) {
+  extern __shared__ uint32_t keys[];  // Np keys, then the per-warp list buffers
+  __shared__ int panel_n[kMaxPanels];
+  const int O = a.O, n = a.n, P = a.P;
+  const int i = blockIdx.x;
+  const uint16_t* row = a.W + (size_t)i * O;
+  uint32_t* lists = keys + a.Np;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+
+  if (threadIdx.x < kMaxPanels) panel_n[threadIdx.x] = 0;
   bool bad = false;
-  for (int j = threadIdx.x; j < Np; j += blockDim.x) {
+  for (int j = threadIdx.x; j < a.Np; j += blockDim.x) {
     uint32_t key = 0xFFFFFFFFu;
     if (j < O) {
       const uint32_t b = row[j];
@@ -60,64 +133,170 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
     }
     keys[j] = key;
   }
-  if (bad) atomicOr(status, kStatusNonfiniteW);
+  if (bad) atomicOr(a.status, kStatusNonfiniteW);
   __syncthreads();
-  bitonic_sort_u32(keys, Np);
+  bitonic_sort_u32(keys, a.Np);
 
   // dense copy of the kept weights (dropped ones stay +0.0 from the memset)
   for (int r = threadIdx.x; r < n; r += blockDim.x) {
     const int j = (int)(keys[r] & 0xFFFFu);
-    wdense[(size_t)i * dstride + j] = row[j];
+    a.wdense[(size_t)i * a.dstride + j] = row[j];
+    atomicAdd(&panel_n[j / kPW], 1);
   }
   if (threadIdx.x < kP) {
-    const int k = threadIdx.x, r = hdp->prank[k];
-    probes[(size_t)i * kP + k] = (r >= 0) ? (uint16_t)(0x7FFFu - (keys[r] >> 16)) : (uint16_t)0;
+    const int r = a.prank[threadIdx.x];
+    a.probes[(size_t)i * kP + threadIdx.x] = (r >= 0) ? (uint16_t)(0x7FFFu - (keys[r] >> 16)) : (uint16_t)0;
   }
-  for (int k = threadIdx.x; k <= C; k += blockDim.x) {
-    const int r = (k == 0) ? 0 : min(k * H, n) - 1;
-    ckmag[(size_t)i * (C + 1) + k] = (uint16_t)(0x7FFFu - (keys[r] >> 16));
-  }
+  __syncthreads();
 
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-  for (int t = warp; t < T; t += nwarps) {
-    int running = 0;
-    const size_t bbase = ((size_t)t * I + i) * kCap;
-    for (int cb = 0; cb < n; cb += 32) {
-      const int r = cb + lane;
-      int j = 0;
-      bool m = false;
-      if (r < n) {
-        j = (int)(keys[r] & 0xFFFFu);
-        m = (j >> 8) == t;
-      }
-      const unsigned bal = __ballot_sync(0xFFFFFFFFu, m);
-      if (m) {
-        const int pos = running + __popc(bal & ((1u << lane) - 1u));
-        vals[bbase + pos] = row[j];
-        idx[bbase + pos] = (uint8_t)(j & 255);
-      }
-      running += __popc(bal);
-      const int end = cb + 32;
-      if (lane == 0 && end <= n && end % H == 0) {
-        cnt[((size_t)i * C + (end / H - 1)) * T + t] = (uint8_t)min(running, 255);
-      }
+  for (int p = warp; p < P; p += kPrepThreads / 32) {
+    uint32_t* list = lists + (size_t)warp * EFFORT_PREP_LIST_MAX;
+    const int pbase = p * kPW;
+    const int np = panel_n[p];
+    const int nstore = (np * kStoreNum + kStoreDen - 1) / kStoreDen;
+    const int want = min(np, nstore + 1);  // stored entries plus the first unstored one
+    // the panel's kept entries in rank order
+    int got = 0;
+    for (int r0 = 0; r0 < n && got < want; r0 += 32) {
+      const int r = r0 + lane;
+      const uint32_t key = (r < n) ? keys[r] : 0xFFFFFFFFu;
+      const bool in = (r < n) && ((int)(key & 0xFFFFu) / kPW == p);
+      const unsigned bal = __ballot_sync(0xFFFFFFFFu, in);
+      const int pos = got + __popc(bal & ((1u << lane) - 1u));
+      if (in && pos < want) list[pos] = key;
+      got += __popc(bal);
     }
-    if (lane == 0 && n % H != 0) cnt[((size_t)i * C + (C - 1)) * T + t] = (uint8_t)min(running, 255);
+    __syncwarp();
+    const unsigned tail = (np > nstore) ? (0x7FFFu - (list[nstore] >> 16)) : 0u;
+    // plan: greedy chunks of at most kCS slots
+    int nchunks = 0;
+    for (int q = 0; q < nstore;) {
+      int t = min(kCS, nstore - q);
+      int s = chunk_slots(list, q, t, pbase);
+      while (s > kCS) {
+        t -= s - kCS;
+        s = chunk_slots(list, q, t, pbase);
+      }
+      q += t;
+      ++nchunks;
+    }
+    unsigned base = 0;
+    if (lane == 0) base = atomicAdd(a.chunk_count, (unsigned)nchunks);
+    base = __shfl_sync(0xFFFFFFFFu, base, 0);
+    if (base + (unsigned)nchunks > a.cap_chunks) {
+      if (lane == 0) atomicOr(a.status, kStatusInternal);
+      continue;
+    }
+    // emit: the same cut again, now writing the slots
+    int k = 0;
+    for (int q = 0; q < nstore; ++k) {
+      int t = min(kCS, nstore - q);
+      int s = chunk_slots(list, q, t, pbase);
+      while (s > kCS) {
+        t -= s - kCS;
+        s = chunk_slots(list, q, t, pbase);
+      }
+      unsigned s0 = (lane < t) ? (list[q + lane] & 0xFFFFu) - pbase : 0xFFFFFFFFu;
+      unsigned s1 = (lane + 32 < t) ? (list[q + lane + 32] & 0xFFFFu) - pbase : 0xFFFFFFFFu;
+      warp_sort64(s0, s1);
+      int g0, g1, f0, f1;
+      chunk_gaps(s0, s1, t, g0, g1, f0, f1);
+      // slot of each entry: entries and fillers before it, plus its own fillers
+      int inc0 = (lane < t) ? 1 + f0 : 0, inc1 = (lane + 32 < t) ? 1 + f1 : 0;
+      int x0 = inc0, x1 = inc1;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y0 = __shfl_up_sync(0xFFFFFFFFu, x0, o), y1 = __shfl_up_sync(0xFFFFFFFFu, x1, o);
+        if (lane >= o) {
+          x0 += y0;
+          x1 += y1;
+        }
+      }
+      const int tot0 = __shfl_sync(0xFFFFFFFFu, x0, 31);
+      x1 += tot0;
+      const int used = __shfl_sync(0xFFFFFFFFu, x1, 31);
+      const size_t slot0 = (size_t)(base + k) * kCS;
+      if (lane < t) {
+        const int e = x0 - inc0;  // first slot of this entry's fillers
+        for (int f = 0; f < f0; ++f) {
+          a.vals[slot0 + e + f] = 0;
+          a.gaps[slot0 + e + f] = 255;
+        }
+        a.vals[slot0 + e + f0] = row[pbase + (int)s0];
+        a.gaps[slot0 + e + f0] = (uint8_t)(g0 - 255 * f0);
+      }
+      if (lane + 32 < t) {
+        const int e = x1 - inc1;
+        for (int f = 0; f < f1; ++f) {
+          a.vals[slot0 + e + f] = 0;
+          a.gaps[slot0 + e + f] = 255;
+        }
+        a.vals[slot0 + e + f1] = row[pbase + (int)s1];
+        a.gaps[slot0 + e + f1] = (uint8_t)(g1 - 255 * f1);
+      }
+      for (int z = used + lane; z < kCS; z += 32) {
+        a.vals[slot0 + z] = 0;
+        a.gaps[slot0 + z] = 0;
+      }
+      if (lane == 0) a.head[base + k] = (uint16_t)(0x7FFFu - (list[q] >> 16));
+      q += t;
+    }
+    if (lane == 0) a.lst[(size_t)i * P + p] = make_uint4(base, (unsigned)nchunks, tail, (unsigned)np);
   }
+}
+
+size_t prep_smem_bytes(int Np) {
+  return (size_t)Np * 4 + (size_t)kMaxPanels * EFFORT_PREP_LIST_MAX * 4;  // list buffers of warps 0..P-1
 }
 
 cudaError_t prep_attributes() {
-  return cudaFuncSetAttribute(k_prep_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, EFFORT_PREP_SMEM_MAX);
+  return cudaFuncSetAttribute(k_prep_rows, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)prep_smem_bytes(EFFORT_PREP_KEYS_MAX));
 }
 
-cudaError_t launch_prep(const uint16_t* W, const HandleDesc* d_desc, int I, int O, uint16_t* vals, uint8_t* idx,
-                        uint16_t* wdense, uint16_t* probes, uint16_t* ckmag, uint8_t* cnt, unsigned int* status,
-                        cudaStream_t stream) {
+cudaError_t launch_prep(const uint16_t* W, int I, int O, int n, int P, int dstride, const int* prank,
+                        uint16_t* wdense, uint16_t* probes, uint16_t* vals, uint8_t* gaps, uint16_t* head, uint4* lst,
+                        unsigned* chunk_count, unsigned cap_chunks, unsigned* status, cudaStream_t stream) {
+  PrepArgs a;
+  a.W = W;
+  a.I = I;
+  a.O = O;
+  a.n = n;
+  a.P = P;
+  a.dstride = dstride;
   int Np = 1;
   while (Np < O) Np <<= 1;
-  const size_t smem = (size_t)Np * 4;
-  k_prep_rows<<<I, kPrepThreads, smem, stream>>>(W, d_desc, Np, vals, idx, wdense, probes, ckmag, cnt, status);
+  a.Np = Np;
+  a.wdense = wdense;
+  a.probes = probes;
+  a.vals = vals;
+  a.gaps = gaps;
+  a.head = head;
+  a.lst = lst;
+  a.chunk_count = chunk_count;
+  a.cap_chunks = cap_chunks;
+  a.status = status;
+  for (int k = 0; k < kP; ++k) a.prank[k] = prank[k];
+  cudaError_t e = prep_attributes();
+  if (e != cudaSuccess) return e;
+  k_prep_rows<<<I, kPrepThreads, prep_smem_bytes(Np), stream>>>(a);
   return cudaGetLastError();
+}
+
+// Upper bound on the chunks of one row: per panel, the stored entries over the
+// fewest entries a full chunk holds (kCS minus the fillers a panel's span can
+// need).
+unsigned long long prep_chunk_bound_per_row(int O, int n) {
+  unsigned long long total = 0;
+  const int P = (O + kPW - 1) / kPW;
+  for (int p = 0; p < P; ++p) {
+    const int w = (p == P - 1) ? O - p * kPW : kPW;
+    const int np = n < w ? n : w;
+    const int nstore = (np * kStoreNum + kStoreDen - 1) / kStoreDen;
+    const int per = kCS - (w / 255 + 1);
+    total += (unsigned long long)((nstore + per - 1) / per);
+  }
+  return total;
 }
 
 }  // namespace effort

@@ -45,7 +45,7 @@ typedef enum {
   EFFORT_ERR_CUDA = 2,         /* a CUDA runtime call or kernel launch failed */
   EFFORT_ERR_NOMEM = 3,        /* device or host allocation failed */
   EFFORT_ERR_NONFINITE = 4,    /* W (prepare) or v (reported by effort_check) held inf/NaN */
-  EFFORT_ERR_DEVICE = 5,       /* a kernel reported an internal inconsistency */
+  EFFORT_ERR_DEVICE = 5,       /* a kernel reported an internal inconsistency or a wait timed out */
   EFFORT_ERR_UNSUPPORTED = 6   /* sizes outside the limits stated below */
 } effort_status_t;
 
@@ -53,8 +53,7 @@ typedef enum { EFFORT_F32 = 0, EFFORT_F16 = 1 } effort_dtype_t;
 
 /* Size limits of this build. */
 #define EFFORT_MAX_OUT_DIM 32768      /* a row is sorted inside one thread block */
-#define EFFORT_MAX_IN_DIM 40960       /* the cutoff's chart lives in one cluster's shared memory */
-#define EFFORT_MAX_PAIRS_PER_LAUNCH 16
+#define EFFORT_MAX_IN_DIM 40960       /* a block's share of the chart lives in its shared memory */
 #define EFFORT_STATIC_SCRATCH_BYTES (2u << 20) /* per-device scratch of effort_gemv_static */
 
 /*
@@ -62,17 +61,21 @@ typedef enum { EFFORT_F32 = 0, EFFORT_F16 = 1 } effort_dtype_t;
  *   Sorts every row of W by |w| descending (ties: lower column first), keeps
  *   the first n = floor(keep_fraction * out_dim + 1/2) entries of each row
  *   (the post text: the format lets the loader skip the least important
- *   weights), takes 16 midpoint-rank probes per row, and stores the kept
- *   entries in output-tile buckets of 256 columns (fp16 value + 8-bit local
- *   index, bucket-sorted by |w|), a dense copy of the kept weights, and the
- *   checkpoint tables the dispatch uses.
+ *   weights), takes 16 midpoint-rank probes per row, and stores, for every row
+ *   and every panel of 2048 output columns, the leading 3/8 of the row's kept
+ *   entries in that panel in rank order, cut into chunks of 64 slots (each
+ *   chunk sorted by column: fp16 value + 8-bit column gap); plus a dense copy
+ *   of the kept weights for rows a call uses beyond that share.
  *   W: device, binary16 [in_dim x out_dim], 2-byte aligned; read only during
  *      the call (the stream is synchronised before returning; the caller may
  *      free W afterwards).
  *   keep_fraction: (0, 1].  Must keep at least one weight per row.
  *   Limits: 1 <= out_dim <= EFFORT_MAX_OUT_DIM, 1 <= in_dim <= EFFORT_MAX_IN_DIM,
  *           in_dim * out_dim < 2^32.
- *   Returns EFFORT_ERR_NONFINITE (and no handle) if W holds inf or NaN.
+ *   Returns EFFORT_ERR_NONFINITE (and no handle) if W holds inf or NaN, and
+ *   EFFORT_ERR_NOMEM if a device allocation fails or would take the library's
+ *   device memory past the cap set by the environment variable
+ *   EFFORT_ALLOC_CAP_BYTES (read at each allocation; unset = no cap).
  *   On success *out_handle owns all device storage; free it with effort_destroy.
  */
 effort_status_t effort_prepare(const void* W, int64_t in_dim, int64_t out_dim, float keep_fraction,
@@ -85,7 +88,12 @@ effort_status_t effort_prepare(const void* W, int64_t in_dim, int64_t out_dim, f
  *   targeted; the cutoff c is the weighted K-th largest entry of the chart
  *   fl32(|v_i| * probe_ik) (c = 0 if K >= the kept count, c = +inf if K = 0).
  *   Asynchronous and stream-ordered: no host synchronisation and no
- *   allocation; two kernels (cutoff+dispatch, then multiply-accumulate).
+ *   allocation; one kernel whose blocks (one per SM) compute the cutoff,
+ *   the dispatch and the multiply-accumulate, meeting at grid-wide barriers.
+ *   out is accumulated in fp32 with reductions whose order varies from call
+ *   to call: c, |S| and the L_i are reproducible bit for bit, out to rounding.
+ *   Each barrier wait has a time limit (0.2 s); a wait that runs out sets a
+ *   status bit that effort_check reports as EFFORT_ERR_DEVICE.
  *   A handle holds one call's scratch: calls on the same handle must be
  *   ordered (same stream, or synchronised); concurrent calls on one handle race.
  */
@@ -107,15 +115,17 @@ effort_status_t effort_gemv_ex(effort_handle_t h, const void* v, effort_dtype_t 
  * effort_gemv_host -- effort_gemv_ex on HOST buffers, for callers that hold v
  *   and want out in host memory.  The pages have no counterpart: this is a
  *   library service around the same matvec.  On `stream`, in order, the same
- *   two kernels as effort_gemv_ex, with v (in_dim elements of v_dtype) and
- *   out (out_dim fp32) moved across the host link as follows:
- *   - page-locked memory mapped into the device's address space (cudaHostAlloc,
- *     cudaMallocHost, cudaHostRegister with mapping; cudaPointerGetAttributes
- *     decides) is read (v) and written (out) in place by the kernels, with no
- *     copy operation;
- *   - other host memory goes through the handle's device staging buffer, with
- *     one cudaMemcpyAsync before the kernels (v) and one after (out); CUDA
- *     stages pageable copies, which may block the host.
+ *   kernel as effort_gemv_ex, with v (in_dim elements of v_dtype) and out
+ *   (out_dim fp32) moved across the host link as follows:
+ *   - v in page-locked memory mapped into the device's address space
+ *     (cudaHostAlloc, cudaMallocHost, cudaHostRegister with mapping;
+ *     cudaPointerGetAttributes decides) is read in place by the kernel; other
+ *     host memory is copied into the handle's device staging buffer with one
+ *     cudaMemcpyAsync before the kernel;
+ *   - out is accumulated in the staging buffer (the kernel adds partial sums
+ *     into it with device-memory reductions) and copied back with one
+ *     cudaMemcpyAsync after the kernel.  CUDA stages copies from or to
+ *     pageable memory, which may block the host.
  *   v_host, out_host: host memory, non-NULL.
  *   The call does not synchronise: out_host holds the result once the stream
  *   has passed this call (cudaStreamSynchronize, an event).  The caller must
@@ -128,17 +138,24 @@ effort_status_t effort_gemv_host(effort_handle_t h, const void* v_host, effort_d
                                  float* out_host, void* stream);
 
 /*
- * effort_gemv_split -- effort_gemv_ex that also records `mid_event` (a
- *   cudaEvent_t passed as void*, created by the caller) on the stream between
- *   the cutoff/dispatch kernel and the multiply kernel, so that each phase can
- *   be timed with events.  The multiply kernel then starts after the event
- *   instead of launching early against the first kernel.  mid_event non-NULL.
- *   Under stream capture the event is recorded with cudaEventRecordExternal,
- *   so that it becomes an event-record node of the CUDA graph.
+ * effort_gemv_timed -- effort_gemv_ex (no optional outputs) that also stores
+ *   the GPU global timer (ns) at fixed points of the call, for per-phase
+ *   timing: marks is a device uint64 array [blocks][16] (blocks from
+ *   effort_grid_blocks); entry k of block b is written by that block when it
+ *   reaches point k: 0 start, 1 after waiting for the preceding grid, 2 chart
+ *   histogram pushed, 3 after the first grid barrier, 4 dispatch bounds
+ *   published, 5 after the second grid barrier, 6 cutoff resolved, 7 work
+ *   range known, 8 first work lists built, 9 first dense units done, 10 first
+ *   round of sparse chunks done, 11 the block's sums added into out, 13 the
+ *   block is done (12 is not used).  Points a call does not reach
+ *   (effort 1 skips 2..5, a tiny effort returns after 1) keep their old
+ *   contents.  The pages have no counterpart: a measurement service.
  */
-effort_status_t effort_gemv_split(effort_handle_t h, const void* v, effort_dtype_t v_dtype, float effort,
-                                  float* out, float* cutoff_out, uint64_t* count_out, void* mid_event,
-                                  void* stream);
+effort_status_t effort_gemv_timed(effort_handle_t h, const void* v, effort_dtype_t v_dtype, float effort,
+                                  float* out, uint64_t* marks, void* stream);
+
+/* Blocks of the grid a matvec on this handle launches (one per SM). */
+effort_status_t effort_grid_blocks(effort_handle_t h, int32_t* blocks);
 
 /*
  * effort_gemv_static -- effort_gemv_ex (without rowlen_out) whose per-call
@@ -151,8 +168,8 @@ effort_status_t effort_gemv_split(effort_handle_t h, const void* v, effort_dtype
  *   front), or that needs its device footprint fixed before the first call.
  *   The call allocates nothing: no cudaMalloc, no cudaFree, no allocating
  *   library routine.  It issues one cudaMemsetAsync that clears the scratch
- *   words that must start at zero, the same two kernels as effort_gemv_ex,
- *   and, if status_out is given, one 4-byte device-to-device copy.
+ *   words that must start at zero, the same kernel as effort_gemv_ex, and,
+ *   if status_out is given, one 4-byte device-to-device copy.
  *   v, v_dtype, effort, out, cutoff_out, count_out: as for effort_gemv_ex.
  *   status_out: nullable device uint32; receives 0 if the call saw only
  *     finite entries of v and no internal inconsistency, nonzero otherwise
@@ -164,8 +181,12 @@ effort_status_t effort_gemv_split(effort_handle_t h, const void* v, effort_dtype
  *     GPU (unordered streams, concurrent host threads) race and give wrong
  *     results; order them on one stream.
  *   Returns EFFORT_ERR_UNSUPPORTED when the handle's geometry needs more than
- *     EFFORT_STATIC_SCRATCH_BYTES of scratch (4096 x 14336 needs about 0.5 MiB,
- *     14336 x 4096 about 0.6 MiB), and when the device ordinal is 64 or above.
+ *     EFFORT_STATIC_SCRATCH_BYTES of scratch (about 60 KiB plus 8 bytes per
+ *     row and 2048-column panel: 4096 x 14336 and 14336 x 4096 need about
+ *     0.3 MiB; in_dim x out_dim / 2048 may reach about 250,000), and when
+ *     the device ordinal is 64 or above.
+ *   The array's address is looked up again whenever the device's primary
+ *     context has changed (after cudaDeviceReset), never kept across it.
  */
 effort_status_t effort_gemv_static(effort_handle_t h, const void* v, effort_dtype_t v_dtype, float effort,
                                    float* out, float* cutoff_out, uint64_t* count_out, uint32_t* status_out,
@@ -174,8 +195,12 @@ effort_status_t effort_gemv_static(effort_handle_t h, const void* v, effort_dtyp
 /*
  * effort_check -- synchronises the handle's last stream and reports whether a
  *   call since the previous check saw a non-finite entry of v
- *   (EFFORT_ERR_NONFINITE; those calls' outputs are unspecified) or an internal
- *   device inconsistency (EFFORT_ERR_DEVICE).  Clears the flags.
+ *   (EFFORT_ERR_NONFINITE; those calls' outputs are unspecified) or a device
+ *   inconsistency: a grid-wide wait that ran out of time, or, in a library
+ *   built with -DEFFORT_DEBUG, an index a kernel found out of range
+ *   (EFFORT_ERR_DEVICE; outputs of the calls since the previous check are
+ *   unspecified).  Clears the flags; after an error it also resets the
+ *   handle's scratch, so that later calls start clean.
  */
 effort_status_t effort_check(effort_handle_t h);
 
@@ -197,8 +222,8 @@ effort_status_t effort_workspace_destroy(effort_workspace_t ws);
  *   HOST arrays of n_pairs entries.  All handles must share in_dim/out_dim
  *   with the workspace.  cutoffs_out [n_pairs] float and counts_out
  *   [n_pairs] uint64 are nullable device arrays.  One cutoff per pair.
- *   Launches two kernels per group of up to EFFORT_MAX_PAIRS_PER_LAUNCH pairs.
- *   n_pairs <= the workspace's max_pairs.
+ *   Launches one kernel per pair, in order on `stream`; the pairs share the
+ *   workspace's scratch.  n_pairs <= the workspace's max_pairs.
  */
 effort_status_t effort_gemv_batched(effort_workspace_t ws, const effort_handle_t* handles, const int32_t* hidx,
                                     const int32_t* vidx, int32_t n_pairs, const void* V, effort_dtype_t v_dtype,
@@ -214,42 +239,62 @@ effort_status_t effort_gemv_batched(effort_workspace_t ws, const effort_handle_t
 effort_status_t effort_dense_gemv(effort_workspace_t ws, const void* W, int64_t in_dim, int64_t out_dim,
                                   const void* v, effort_dtype_t v_dtype, float* out, void* stream);
 
-/* Sizes and footprint of a prepared matrix. */
+/* Sizes and footprint of a prepared matrix (device_bytes: its stored format,
+ * not counting the per-call scratch and staging buffer). */
 effort_status_t effort_get_info(effort_handle_t h, int64_t* in_dim, int64_t* out_dim, float* keep_fraction,
                                 size_t* device_bytes);
 
 /*
  * effort_layout_t -- read-only view of a handle's device storage, for format
- * checks.  Bucket (i, t) holds the kept entries of row i with columns in
- * [256 t, 256 t + 256), sorted by |w| descending (ties: lower column), at
- * entry offset (t * in_dim + i) * bucket_cap of `vals` (binary16 bits) and
- * `idx` (column - 256 t); unused slots hold +0.0 / 0.
- * probes: [in_dim][16] |w| binary16 bits at the probe ranks (0 for empty segments).
- * ckmag: [in_dim][n_ck + 1]: [0] = |w| at rank 0; [1 + k] = |w| at rank
- *   min((k + 1) * ck_step, n) - 1.
- * cnt: [in_dim][n_ck][n_tiles] uint8: entries of tile t among the first
- *   min((k + 1) * ck_step, n) ranks of row i, saturated at 255.
- * wdense: [in_dim][n_tiles * 256] binary16: kept weights at their columns, 0 elsewhere.
- * rec / gcnt: the last call's dispatch records (see the library source).
+ * checks.  Panel p covers columns [panel_width p, panel_width (p + 1)).
+ * lists: [in_dim][n_panels] of {first chunk, stored chunks, tail, kept}: list
+ *   (i, p) holds the kept entries of row i in panel p in row i's order (|w|
+ *   descending, ties: lower column); its leading ceil(kept * store_num /
+ *   store_den) entries are stored in chunks [first, first + stored chunks);
+ *   tail is the |w| binary16 bits of the first entry not stored (0 if none).
+ * vals / gaps: chunk c occupies slots [chunk_slots c, chunk_slots (c + 1)):
+ *   binary16 value bits and 8-bit column gaps.  The slots of a chunk are in
+ *   column order; the column of a slot is -1 + the sum of the gaps up to and
+ *   including it (panel-local).  Filler slots (value +0, gap 255) bridge gaps
+ *   above 255; pad slots (value +0, gap 0) fill the chunk.
+ * head: [total_chunks] |w| bits of each chunk's first (largest) rank.
+ * wdense: [in_dim][dense_stride] binary16: kept weights at their columns, +0
+ *   elsewhere.  probes: [in_dim][16] |w| bits at the probe ranks (0 for empty
+ *   segments).  scratch_bytes: the handle's per-call scratch.
  */
 typedef struct {
   int64_t in_dim, out_dim;
-  int32_t n_kept, n_tiles, bucket_cap, ck_step, n_ck, n_probes;
+  int32_t n_kept, n_panels, panel_width, chunk_slots, store_num, store_den, n_probes, dense_stride;
+  uint32_t total_chunks;
   const void* vals;
-  const void* idx;
-  const void* probes;
-  const void* ckmag;
-  const void* cnt;
+  const void* gaps;
+  const void* head;
+  const void* lists;
   const void* wdense;
-  const void* rec;
-  const void* gcnt;
-  int32_t n_groups;
+  const void* probes;
+  size_t scratch_bytes;
 } effort_layout_t;
 
 effort_status_t effort_get_layout(effort_handle_t h, effort_layout_t* layout);
 
 /* Frees the handle's device storage after synchronising its last stream. */
 effort_status_t effort_destroy(effort_handle_t h);
+
+/*
+ * effort_last_call_bytes -- the bytes of the prepared matrix that the handle's
+ *   last finished call (effort_gemv, _ex, _host) planned to read: dense_bytes
+ *   for the (row, panel) units it read from the dense copy (512 bytes per
+ *   256-column stripe), sparse_bytes for the chunks (3 bytes per slot, 64
+ *   slots per chunk).  Synchronises the handle's last stream.  The pages have
+ *   no counterpart: a measurement service.  dense_bytes, sparse_bytes: host
+ *   pointers, non-NULL.
+ */
+effort_status_t effort_last_call_bytes(effort_handle_t h, uint64_t* dense_bytes, uint64_t* sparse_bytes);
+
+/* Device memory the library holds at this moment, over all handles and
+ * workspaces of the process (the figure EFFORT_ALLOC_CAP_BYTES is checked
+ * against).  bytes: host pointer, non-NULL. */
+effort_status_t effort_device_bytes_held(uint64_t* bytes);
 
 /* Static string naming a status code. */
 const char* effort_status_string(effort_status_t s);

@@ -12,12 +12,36 @@ import bench  # noqa: E402
 
 
 def test_traffic_record_is_dropped_once_the_sources_change(monkeypatch):
-    rec = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))["k_mac"]
+    recs = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))
+    name, rec = next(iter(recs.items()))
     monkeypatch.setattr(bench, "source_sha", lambda *names: rec["source_sha"])
-    assert bench.ncu_traffic("k_mac") == float(rec["dram_bytes_per_launch"])
+    assert bench.ncu_traffic(name) == float(rec["dram_bytes_per_launch"])
     monkeypatch.setattr(bench, "source_sha", lambda *names: "0" * 16)
-    assert bench.ncu_traffic("k_mac") is None
+    assert bench.ncu_traffic(name) is None
     assert bench.ncu_traffic("no_such_kernel") is None
+
+
+def test_reference_arm_labels_a_row_slice_as_extrapolated(monkeypatch, capsys):
+    """When whole oracle matvecs would not fit the run's time budget, each step
+    is a row slice, value is scaled to the full matvec, ms_per_step stays the
+    time a step really took, and the line says so."""
+    import numpy as np
+    import argparse
+    monkeypatch.setattr(bench, "oracle_workload", lambda rows=bench.IN_DIM, seed=4, n_vecs=4: (None, rows, [None]))
+    calls = []
+
+    def fake_time(prep, vs, min_calls, budget_s=0.0):
+        calls.append((prep, min_calls))
+        return (10.0 if prep == bench.IN_DIM else 10.0 * prep / bench.IN_DIM), max(min_calls, 1), 1.0
+
+    monkeypatch.setattr(bench, "time_oracle_calls", fake_time)
+    monkeypatch.delenv("RANK", raising=False)
+    bench.run_reference(argparse.Namespace(steps=2000, warmup=200, gpus=1))
+    d = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    ex = d["extrapolated"]
+    assert ex is not None and ex["rows_per_step"] < bench.IN_DIM
+    assert np.isclose(d["value"], d["ms_per_step"] * 1e3 * ex["scale_to_full_matvec"])
+    assert d["ms_per_step"] * d["steps"] / 1e3 <= bench.REFERENCE_BUDGET_S * 1.01
 
 
 def test_reference_arm_prints_one_contract_line():

@@ -9,6 +9,9 @@ Contract per call, on seeded synthetic inputs:
     product by product);
   * out agrees with the oracle's float64 sum over the same set to relative
     L2 <= 1e-4 and max abs error <= 1e-3 * ||out||_inf.
+The cutoff, |S| and the L_i are also identical from call to call.  out is
+summed in fp32 with shared-memory atomics, whose order varies, so repeated
+calls agree to rounding (checked at relative L2 1e-6), not bit for bit.
 """
 import numpy as np
 import pytest
@@ -81,39 +84,101 @@ def make(E, I, Od, seed, keep=1.0):
 
 
 # ------------------------------------------------------------------ format
+def decode_chunk(vals, gaps, c, cs):
+    """(column, value bits, kind) of the slots of chunk c; kind is 'entry',
+    'filler' (value +0, gap 255) or 'pad' (value +0, gap 0, after the entries)."""
+    v = vals[c * cs:(c + 1) * cs].view(np.uint16).astype(np.int64)
+    g = gaps[c * cs:(c + 1) * cs].astype(np.int64)
+    cols = -1 + np.cumsum(g)
+    kinds = []
+    for s_ in range(cs):
+        if v[s_] != 0:
+            kinds.append("entry")
+        elif g[s_] == 255:
+            kinds.append("filler")
+        else:
+            kinds.append("pad")
+    return cols, v, kinds
+
+
 def check_layout(prep, pm):
     L = {k: (v.cpu().numpy() if isinstance(v, torch.Tensor) else v) for k, v in pm.layout().items()}
     I, Od, n = prep.in_dim, prep.out_dim, prep.n
-    T, H, C = L["n_tiles"], L["ck_step"], L["n_ck"]
-    assert L["n_kept"] == n
+    P, PW, cs = L["n_panels"], L["panel_width"], L["chunk_slots"]
+    assert L["n_kept"] == n and P == (Od + PW - 1) // PW
     Wb = prep.W_bits
+    seen = np.zeros(L["total_chunks"], dtype=bool)
     for i in range(I):
         order = prep.W_idx[i, :n]
-        tiles = order // 256
-        for t in range(T):
-            cols = order[tiles == t]
-            nb = cols.size
-            assert np.array_equal(L["vals"][t, i, :nb].view(np.uint16), Wb[i, cols])
-            assert np.array_equal(L["idx"][t, i, :nb], (cols - 256 * t).astype(np.uint8))
-            assert not np.any(L["vals"][t, i, nb:]) and not np.any(L["idx"][t, i, nb:])
-            for k in range(C):
-                end = min((k + 1) * H, n)
-                assert L["cnt"][i, k, t] == min(255, int(np.sum(tiles[:end] == t)))
-        mag = (Wb[i, order] & 0x7FFF)
+        mag = (Wb[i] & 0x7FFF).astype(np.int64)
+        for p in range(P):
+            first, S, tail, kept = (int(x) for x in L["lists"][i, p])
+            cols = order[order // PW == p]              # the list: panel p's kept entries in row order
+            assert kept == cols.size
+            nstore = (3 * kept + 7) // 8
+            assert tail == (mag[cols[nstore]] if kept > nstore else 0)
+            got = []
+            for k in range(S):
+                c = first + k
+                assert not seen[c]
+                seen[c] = True
+                ccols, cv, kinds = decode_chunk(L["vals"], L["gaps"], c, cs)
+                ent = [s_ for s_ in range(cs) if kinds[s_] == "entry"]
+                # slots in column order, pads only after the last entry, fillers before an entry
+                assert np.all(np.diff(ccols[ent]) > 0)
+                last = ent[-1]
+                assert all(kd == "pad" for kd in kinds[last + 1:])
+                assert all(kd != "pad" for kd in kinds[:last])
+                assert ccols[0] >= 0 and ccols[last] < min(PW, Od - p * PW)
+                chunk_cols = ccols[ent] + p * PW
+                assert np.array_equal(cv[ent], Wb[i, chunk_cols])
+                # a chunk is a run of consecutive ranks: its entries are the next ones of the list
+                run = cols[len(got):len(got) + len(ent)]
+                assert np.array_equal(np.sort(run), chunk_cols)
+                assert int(L["head"][c]) & 0xFFFF == mag[run[0]]
+                if k < S - 1:
+                    assert kinds.count("pad") == 0  # the greedy cut fills every chunk but the last
+                got.extend(run.tolist())
+            assert len(got) == nstore
         ranks, weights = O.probe_layout(n)
-        exp_probes = np.where(weights > 0, mag[np.maximum(ranks, 0)], 0)
+        srt = mag[order]
+        exp_probes = np.where(weights > 0, srt[np.maximum(ranks, 0)], 0)
         assert np.array_equal(L["probes"][i].view(np.uint16), exp_probes)
-        ck = [mag[0]] + [mag[min((k + 1) * H, n) - 1] for k in range(C)]
-        assert np.array_equal(L["ckmag"][i].view(np.uint16), np.array(ck, np.uint16))
-        dense = np.zeros(T * 256, np.uint16)
+        dense = np.zeros(L["dense_stride"], np.uint16)
         dense[order] = Wb[i, order]
         assert np.array_equal(L["wdense"][i].view(np.uint16), dense)
+    assert seen.all()
 
 
-@pytest.mark.parametrize("I,Od,keep", [(40, 300, 1.0), (33, 513, 0.75), (7, 9, 1.0), (64, 1024, 0.8)])
+@pytest.mark.parametrize("I,Od,keep", [(40, 300, 1.0), (33, 513, 0.75), (7, 9, 1.0), (24, 5000, 0.8),
+                                       (6, 14336, 1.0)])
 def test_layout_matches_oracle_order(E, I, Od, keep):
     _, prep, pm = make(E, I, Od, 101, keep)
     check_layout(prep, pm)
+
+
+def test_layout_fillers_bridge_wide_gaps(E):
+    """Rows whose consecutive ranks sit far apart in column: |w_ij| falls with
+    j mod 300, so a chunk's run of ranks takes a few residues from every
+    300-column stretch and its sorted columns jump by about 290, which filler
+    slots bridge."""
+    I, Od = 4, 4096
+    j = np.arange(Od)
+    sign = np.where(inputs.weights(I, Od, 5) < 0, -1.0, 1.0)
+    Wn = (sign * (1.0 - (j % 300) / 1000.0)[None, :]).astype(np.float16)
+    prep = O.Prepared(Wn.view(np.uint16), 1.0)
+    pm = E.PreparedMatrix(torch.from_numpy(Wn).cuda(), 1.0)
+    check_layout(prep, pm)
+    g = pm.layout()["gaps"].cpu().numpy()
+    assert np.any(g == 255)
+
+
+def test_storage_within_1_6x_of_fp16(E):
+    """The stored format (chunks, dense copy, tables) stays within 1.6x the
+    fp16 bytes of W at keep 1."""
+    _, prep, pm = make(E, 1024, 14336, 3)
+    info = pm.info()
+    assert info["device_bytes"] <= 1.6 * 2 * 1024 * 14336
 
 
 # ------------------------------------------------------------------ parity
@@ -177,14 +242,13 @@ def test_host_buffers_match_device_call(E, dtype):
     out_host = torch.full((1300,), float("nan"), dtype=torch.float32).pin_memory()
     pm.gemv_host(v_host, 0.3, out_host)
     torch.cuda.synchronize()
-    dev_out = pm.gemv(torch.from_numpy(v_np).cuda(), 0.3).cpu()
-    assert torch.equal(out_host, dev_out)
-    assert_out_close(out_host.numpy(), O.effort_gemv(prep, v_np, 0.3).out)
+    ref = O.effort_gemv(prep, v_np, 0.3).out
+    assert_out_close(out_host.numpy(), ref)
     # pageable host memory goes through the staging buffer and copies
     out2 = torch.zeros(1300, dtype=torch.float32)
     pm.gemv_host(torch.from_numpy(v_np), 0.3, out2)
     torch.cuda.synchronize()
-    assert torch.equal(out2, dev_out)
+    assert_out_close(out2.numpy(), ref)
     # pinned buffers are read and written in place: new contents of the same
     # buffers between calls are seen, call after call
     for seed in (23, 24, 25):
@@ -192,7 +256,7 @@ def test_host_buffers_match_device_call(E, dtype):
         v_host.copy_(torch.from_numpy(w_np))
         pm.gemv_host(v_host, 0.3, out_host)
         torch.cuda.synchronize()
-        assert torch.equal(out_host, pm.gemv(torch.from_numpy(w_np).cuda(), 0.3).cpu())
+        assert_out_close(out_host.numpy(), O.effort_gemv(prep, w_np, 0.3).out)
 
 
 def test_one_hot_rows_product_by_product(E):
@@ -207,18 +271,27 @@ def test_one_hot_rows_product_by_product(E):
         assert np.array_equal(out, exp.astype(np.float32))
 
 
-def test_repeat_calls_are_deterministic(E):
+def close_run_to_run(a, b, rel=1e-6):
+    a = a.double().cpu().numpy()
+    b = b.double().cpu().numpy()
+    assert np.linalg.norm(a - b) <= rel * np.linalg.norm(b)
+
+
+def test_repeat_calls_agree(E):
+    """c, |S| and every L_i are identical call after call; out to rounding."""
     _, prep, pm = make(E, 1024, 1536, 14)
     v = torch.from_numpy(inputs.vector(1024, 15, "t3")).cuda()
-    first = pm.gemv(v, 0.25).clone()
+    c0, n0, L0, o0 = run_gpu(E, pm, v, 0.25)
     for _ in range(5):
-        assert torch.equal(pm.gemv(v, 0.25), first)
+        c1, n1, L1, o1 = run_gpu(E, pm, v, 0.25)
+        assert f32bits(c1) == f32bits(c0) and n1 == n0 and np.array_equal(L1, L0)
+        close_run_to_run(torch.from_numpy(o1), torch.from_numpy(o0))
 
 
 def test_back_to_back_calls_on_one_handle(E):
     """Calls queued back to back on one handle and stream, with no host sync:
-    each call's cutoff starts during the previous call's multiply and reuses
-    its scratch.  Every output must equal the same call made alone."""
+    each call's blocks start as the previous call's blocks leave and reuse its
+    scratch.  Every output must match the same call made alone (to rounding)."""
     _, prep, pm = make(E, 2048, 3072, 31)
     vs = [torch.from_numpy(inputs.vector(2048, 40 + k, "t3" if k % 2 else "normal")).cuda() for k in range(4)]
     efforts = [0.25, 0.1, 0.5, 0.25, 1.0, 0.05, 0.3, 0.25]
@@ -232,7 +305,7 @@ def test_back_to_back_calls_on_one_handle(E):
             pm.gemv(vs[k % 4], e, out=outs[k])
         torch.cuda.synchronize()
         for k in range(len(efforts)):
-            assert torch.equal(outs[k], alone[k]), (rep, k)
+            close_run_to_run(outs[k], alone[k])
     ref = O.effort_gemv(prep, vs[1].cpu().numpy(), efforts[1])
     assert_out_close(alone[1].cpu().numpy(), ref.out)
 

@@ -1,8 +1,8 @@
 """effort_gemv_static, the entry point whose scratch is the library's fixed
 per-device array, against effort_gemv_ex on the same handle and inputs.
 
-Both run the same two kernels, so cutoff and |S| must agree bit for bit and
-out within the parity tolerance of the other GPU tests.  Two static calls run
+Both run the same kernel, so cutoff and |S| must agree bit for bit and out
+within the parity tolerance of the other GPU tests.  Two static calls run
 back to back (different vectors and efforts) to show that the words the call
 clears at its start leave no state behind.  This file is collected last so
 that it also runs after every other test in the same process; it passes
@@ -101,7 +101,7 @@ def test_static_reports_nonfinite_v(E):
 def test_static_rejects_geometry_beyond_its_scratch(E):
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
-    I, Od = 40960, 16384  # the read-bound table alone (2.6 MB) exceeds the fixed scratch
+    I, Od = 40960, 16384  # the per-(row, panel) dispatch tables alone (2.6 MB) exceed the fixed scratch
     W = torch.randn(I, Od, device="cuda", dtype=torch.float32).mul_(0.02).half()
     pm = E.PreparedMatrix(W, 1.0)
     del W
