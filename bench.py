@@ -4,10 +4,13 @@
 Headline workload: one approximate matvec out = W^T v with W 4096 x 14336 fp16
 (Mistral-7B FFN w1/w3 shape, entries N(0, 0.02^2)), v fp32 Student-t(3) /
 sqrt(3), effort 0.25, keep 1.0, batch 1.  A step is one call of the library's
-gemv (cutoff + dispatch kernel, then multiply kernel) on inputs resident in
+gemv (one fused kernel: cutoff, dispatch and multiply) on inputs resident in
 HBM.  Steps rotate over 10 prepared matrices and 8 vectors, so the bytes a
 call reads are not in L2 from the previous use.  Steps are issued from CUDA
-graphs (Python launch overhead would otherwise dominate a ~10 us call).
+graphs (Python launch overhead would otherwise dominate a call of tens of
+microseconds).  The timed region of exactly --steps steps is repeated
+TIMED_REGIONS times; the line reports the median region (all of them are
+listed).
 
 Prints ONE JSON line (rank 0).  `--impl reference` times the CPU oracle
 instead (the reference arm).  `--gpus N` under torchrun runs N independent
@@ -33,6 +36,7 @@ METRIC = "approx-GEMV µs & achieved HBM GB/s vs effort (4096×14336 fp16, batch
 IN_DIM, OUT_DIM = 4096, 14336
 EFFORT, KEEP = 0.25, 1.0
 N_MATS, N_VECS, GRAPH_STEPS = 10, 8, 40
+TIMED_REGIONS = 5
 SWEEP = (1.0, 0.5, 0.4, 0.25, 0.15)
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
@@ -65,7 +69,8 @@ def workload_config():
                         f"effort {EFFORT}, keep {KEEP}, batch 1",
             "in_dim": IN_DIM, "out_dim": OUT_DIM, "effort": EFFORT, "keep_fraction": KEEP,
             "l2": f"inputs larger than L2: {N_MATS} prepared matrices x {N_VECS} vectors rotated",
-            "issue": f"CUDA graphs of {GRAPH_STEPS} steps"}
+            "issue": f"CUDA graphs of {GRAPH_STEPS} steps",
+            "timing": f"median of {TIMED_REGIONS} timed regions of --steps steps each"}
 
 
 # ----------------------------------------------------------------- CPU oracle
@@ -234,6 +239,21 @@ def run_reference(a):
     print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------- bytes
+def algorithmic_bytes(in_dim, out_dim, used, v_bytes=4):
+    """Algorithmic bytes of one matvec: 3 bytes per used product (fp16 value
+    and an 8-bit position), the 16 fp16 probes of every row, v and out."""
+    return 3.0 * used + 2.0 * 16 * in_dim + v_bytes * in_dim + 4.0 * out_dim
+
+
+def read_bytes(in_dim, out_dim, dense, sparse, v_bytes=4):
+    """Bytes a call plans to read from the prepared matrix (whole dense
+    panel rows at 2 bytes per entry, stored chunks at 3 bytes per slot), plus
+    probes, v and out: what the kernel actually moves, which unlike the
+    algorithmic figure cannot exceed a copy's bandwidth."""
+    return float(dense) + float(sparse) + 2.0 * 16 * in_dim + v_bytes * in_dim + 4.0 * out_dim
+
+
 # ----------------------------------------------------------------- other shapes
 def measure_shape(E, dev, in_dim, out_dim, efforts, dist, n_mats=10, n_vecs=8, seed0=5000, keep=1.0):
     """us per matvec and algorithmic GB/s on another workload shape: n_mats
@@ -254,11 +274,16 @@ def measure_shape(E, dev, in_dim, out_dim, efforts, dist, n_mats=10, n_vecs=8, s
     res = {}
     steps = 40
     for e in efforts:
-        used = 0.0
+        used, dense, sparse = 0.0, 0.0, 0.0
         for k in range(steps):
             mats[k % n_mats].gemv(vecs[k % n_vecs], e, out=outs[k % n_mats], count=cnt)
             used += float(cnt.item())
+            d, sp = mats[k % n_mats].last_call_bytes()
+            dense += d
+            sparse += sp
         used /= steps
+        dense /= steps
+        sparse /= steps
         s = torch.cuda.Stream(device=dev)
         s.wait_stream(torch.cuda.current_stream(dev))
         gr = torch.cuda.CUDAGraph()
@@ -280,9 +305,12 @@ def measure_shape(E, dev, in_dim, out_dim, efforts, dist, n_mats=10, n_vecs=8, s
         e1.record()
         torch.cuda.synchronize()
         us = e0.elapsed_time(e1) * 1000.0 / (reps * steps)
-        b = 3.0 * used + 4.0 * in_dim + 4.0 * out_dim
+        b = algorithmic_bytes(in_dim, out_dim, used)
+        rb = read_bytes(in_dim, out_dim, dense, sparse)
         dense_b = 2.0 * in_dim * out_dim + 4.0 * in_dim + 4.0 * out_dim
         res[str(e)] = {"us": us, "gbs_algorithmic": b / (us * 1e-6) / 1e9, "mean_used": used,
+                       "read_bytes": {"dense": dense, "sparse": sparse, "total": rb},
+                       "gbs_read": rb / (us * 1e-6) / 1e9,
                        "dense_roofline_us_measured_peak": dense_b / (hbm_peak()[0] * 1e9) * 1e6}
         del gr
     for m in mats:
@@ -570,15 +598,20 @@ def main():
     def step_pairs(n, offset=0):
         return [((offset + k) % N_MATS, (offset + k) % N_VECS) for k in range(n)]
 
-    # used-product counts of the rotation at each effort (algorithmic bytes)
-    def mean_count(effort):
+    # per-step means over the rotation at one effort: used products, and the
+    # bytes each call planned to read per path (dense rows, stored chunks)
+    def rotation_stats(effort):
         cnt = torch.zeros(1, device=dev, dtype=torch.int64)
-        tot = 0
+        used, dense, sparse = 0, 0, 0
         pairs = step_pairs(GRAPH_STEPS)
         for (mi, vi) in pairs:
             mats[mi].gemv(vecs[vi], effort, out=outs[mi], count=cnt)
-            tot += int(cnt.item())
-        return tot / len(pairs)
+            used += int(cnt.item())
+            d, sp = mats[mi].last_call_bytes()
+            dense += d
+            sparse += sp
+        n = len(pairs)
+        return used / n, dense / n, sparse / n
 
     def capture(n_steps, effort, offset=0):
         gr = torch.cuda.CUDAGraph()
@@ -595,25 +628,30 @@ def main():
         torch.cuda.synchronize()
         return gr
 
-    def timed_steps(effort, steps, warmup, sampler=None, min_seconds=0.0):
+    def timed_steps(effort, steps, warmup, regions=1, sampler=None, min_seconds=0.0):
+        """Times `regions` back-to-back regions of exactly `steps` steps (after
+        `warmup` untimed ones); returns each region's milliseconds (max over
+        ranks)."""
         full = capture(GRAPH_STEPS, effort)
         rem = steps % GRAPH_STEPS
         tail = capture(rem, effort, offset=0) if rem else None
         for _ in range(max(1, math.ceil(warmup / GRAPH_STEPS))):
             full.replay()
         torch.cuda.synchronize()
-        barrier()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for _ in range(steps // GRAPH_STEPS):
-            full.replay()
-        if tail is not None:
-            tail.replay()
-        e1.record()
-        torch.cuda.synchronize()
-        barrier()
-        ms = rank_max(e0.elapsed_time(e1))
+        out_ms = []
+        for _ in range(regions):
+            barrier()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(steps // GRAPH_STEPS):
+                full.replay()
+            if tail is not None:
+                tail.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            barrier()
+            out_ms.append(rank_max(e0.elapsed_time(e1)))
         # keep the same replay running until the clock sampler has a window of samples
         if sampler is not None and min_seconds > 0:
             t0 = time.perf_counter()
@@ -621,26 +659,56 @@ def main():
                 for _ in range(50):
                     full.replay()
                 torch.cuda.synchronize()
-        return ms
+        return out_ms
+
+    def phase_marks(effort, calls=12):
+        """Medians (over calls, of the median over blocks) of the fused
+        kernel's phase marks, in microseconds after the earliest block passed
+        its wait on the preceding grid; one call at a time."""
+        nb = mats[0].grid_blocks()
+        marks = torch.zeros(nb, 16, dtype=torch.int64, device=dev)
+        rows = []
+        for k in range(calls):
+            marks.zero_()
+            mats[k % N_MATS].gemv_timed(vecs[k % N_VECS], effort, outs[0], marks)
+            torch.cuda.synchronize()
+            m = marks.cpu().numpy().astype(np.int64)
+            rows.append(m - m[:, 1].min())
+        R = np.stack(rows)
+        names = {0: "start", 1: "wait", 2: "chart_histogram", 3: "barrier_B1", 4: "candidates", 5: "barrier_B2",
+                 6: "cutoff", 7: "dispatch", 8: "dense_streamed", 9: "sparse_streamed", 10: "accumulated",
+                 11: "out_reduced", 13: "end"}
+        res = {}
+        for k, nm in names.items():
+            col = R[:, :, k]
+            if (col == 0).all() or (col < -10 ** 12).any():
+                continue
+            res[nm] = round(float(np.median(np.median(col.astype(np.float64), 1))) / 1e3, 2)
+        return res
 
     peak, peak_kind = hbm_peak()
     sampler = ClockSampler(local)
     sampler.start()
     time.sleep(0.3)
-    ms = timed_steps(EFFORT, a.steps, a.warmup, sampler, min_seconds=2.0)
+    region_ms = timed_steps(EFFORT, a.steps, a.warmup, regions=TIMED_REGIONS, sampler=sampler, min_seconds=2.0)
     clocks = sampler.stop()
+    ms = statistics.median(region_ms)
     us_per_step = ms * 1000.0 / a.steps
     value = whole_job_us_per_matvec(us_per_step, world)
 
-    S_mean = mean_count(EFFORT)
-    alg_bytes = 3.0 * S_mean + 4.0 * IN_DIM + 4.0 * OUT_DIM  # 3-byte entries of the used set + v + out
+    S_mean, D_mean, Sp_mean = rotation_stats(EFFORT)
+    alg_bytes = algorithmic_bytes(IN_DIM, OUT_DIM, S_mean)
+    rd_bytes = read_bytes(IN_DIM, OUT_DIM, D_mean, Sp_mean)
     launch_us = us_per_step  # one kernel per call
     achieved = alg_bytes / (launch_us * 1e-6) / 1e9
     traffic = ncu_traffic("k_effort")
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                 "traffic": traffic, "kernel": "k_effort", "peak_kind": peak_kind,
                 "frac_of_nominal_8000": achieved / NOMINAL_HBM_GBS,
-                "algorithmic_bytes_per_launch": alg_bytes, "launch_us": launch_us}
+                "algorithmic_bytes_per_launch": alg_bytes, "launch_us": launch_us,
+                "read_bytes_per_launch": {"dense": D_mean, "sparse": Sp_mean, "total": rd_bytes},
+                "read_gbs": rd_bytes / (launch_us * 1e-6) / 1e9}
+    phases = phase_marks(EFFORT) if world == 1 else {}
 
     # dense baselines on the same rotation (raw fp16 matrices, 117 MB each)
     ws = E.Workspace(IN_DIM, OUT_DIM)
@@ -687,11 +755,14 @@ def main():
     sweep = {}
     if not a.no_sweep:
         for e in SWEEP:
-            msw = timed_steps(e, 400, 80)
+            msw = statistics.median(timed_steps(e, 400, 80, regions=3))
             us = msw * 1000.0 / 400
-            Se = mean_count(e)
-            b = 3.0 * Se + 4.0 * IN_DIM + 4.0 * OUT_DIM
+            Se, De, Spe = rotation_stats(e)
+            b = algorithmic_bytes(IN_DIM, OUT_DIM, Se)
+            rb = read_bytes(IN_DIM, OUT_DIM, De, Spe)
             sweep[str(e)] = {"us": us, "gbs_algorithmic": b / (us * 1e-6) / 1e9, "mean_used": Se,
+                             "read_bytes": {"dense": De, "sparse": Spe, "total": rb},
+                             "gbs_read": rb / (us * 1e-6) / 1e9,
                              "vs_dense_roofline_measured": baselines["dense_roofline_us_measured_peak"] / us}
 
     # batched / MoE: 8 experts of the workload's shape (the first eight prepared
@@ -718,7 +789,7 @@ def main():
                 used = float(cnt_d.sum().item())
                 ms_call = time_graph(lambda: E.gemv_batched(ws_moe, mats[:n_exp], hidx, vidx, Vd, [e] * (2 * nv),
                                                             OUT=OUTd), n_rep=20)
-                b = 3.0 * used + 2 * nv * (4.0 * IN_DIM + 4.0 * OUT_DIM)
+                b = 3.0 * used + 2 * nv * (algorithmic_bytes(IN_DIM, OUT_DIM, 0.0))
                 row[str(e)] = {"us_per_call": ms_call * 1000.0, "pairs": 2 * nv,
                                "gbs_algorithmic": b / (ms_call * 1e-3) / 1e9}
             moe[str(nv)] = row
@@ -764,6 +835,8 @@ def main():
                 "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
                 "config": workload_config(),
                 "gbs": alg_bytes / (us_per_step * 1e-6) / 1e9,
+                "timed_regions_us_per_step": [x * 1000.0 / a.steps for x in region_ms],
+                "phases_us": phases,
                 "roofline": roofline, "cpu_baseline": cpu,
                 "e2e": {"value": e2e_us, "unit": "us", "h2d_bytes_per_step": 4 * IN_DIM,
                         "d2h_bytes_per_step": 4 * OUT_DIM},

@@ -98,9 +98,8 @@ effort_status_t make_geometry(int64_t I, int64_t O, int n, Geometry* g) {
   g->P = (int)((O + kPW - 1) / kPW);
   g->dstride = (int)((O + kStripe - 1) / kStripe * kStripe);
   g->T = (int)((O + 255) / 256);
-  size_t oc, oh, ocd, ol, octl;
   g->nb = sms;
-  g->smem = smem_layout(g->I, g->nb, &oc, &oh, &ocd, &ol, &octl);
+  g->smem = smem_layout(g->I, g->nb).total;
   if (g->smem > (size_t)optin) return EFFORT_ERR_UNSUPPORTED;
   if (effort_kernel_attributes(g->smem) != cudaSuccess) {
     cudaGetLastError();
@@ -120,8 +119,7 @@ size_t scratch_bytes(const Geometry& g) {
   return align_up((size_t)kHdrWords * 4 + 16, 256)                 // header, barrier, count
          + align_up((size_t)(kBins0 + kBins1 + kBins2) * 4, 256)   // histograms
          + align_up((size_t)kCandCap * 8, 256)                     // candidates
-         + 2 * align_up((size_t)g.I * g.P * 4, 256)                // info, rowpre
-         + align_up((size_t)g.nb * g.P * 4, 256);                  // block totals
+         ;
 }
 // Bytes that must be zero before the first call (header and histograms).
 size_t scratch_zero_bytes() {
@@ -139,12 +137,7 @@ WsPtrs carve(char* b, const Geometry& g) {
   w.ghist2 = w.ghist1 + kBins1;
   b += align_up((size_t)(kBins0 + kBins1 + kBins2) * 4, 256);
   w.cand = (uint2*)b;
-  b += align_up((size_t)kCandCap * 8, 256);
-  w.info = (unsigned*)b;
-  b += align_up((size_t)g.I * g.P * 4, 256);
-  w.rowpre = (unsigned*)b;
-  b += align_up((size_t)g.I * g.P * 4, 256);
-  w.ctot = (unsigned*)b;
+  (void)g;
   return w;
 }
 
@@ -343,7 +336,7 @@ effort_status_t effort_prepare(const void* W, int64_t in_dim, int64_t out_dim, f
   d.lst = (const uint4*)tb;
   d.wdense = (const uint16_t*)(tb + sz_lst);
   d.probes = (const uint16_t*)(tb + sz_lst + sz_dense);
-  unsigned* ctl = (unsigned*)(tb + sz_lst + sz_dense + sz_probe);  // [0] chunk counter, [1] status
+  unsigned* ctl = (unsigned*)(tb + sz_lst + sz_dense + sz_probe);  // [0] chunk counter, [1] max |w| bits, [2] status
   uint16_t* tvals = (uint16_t*)tmp.p;
   uint8_t* tgaps = (uint8_t*)(tvals + (size_t)cap_chunks * kCS);
   uint16_t* thead = (uint16_t*)(tgaps + (size_t)cap_chunks * kCS);
@@ -353,13 +346,14 @@ effort_status_t effort_prepare(const void* W, int64_t in_dim, int64_t out_dim, f
   cudaError_t e = cudaMemsetAsync(h->tables.p, 0, sz_tables, s);
   if (e == cudaSuccess)
     e = launch_prep((const uint16_t*)W, I, O, n, P, dstride, prank, (uint16_t*)d.wdense, (uint16_t*)d.probes, tvals,
-                    tgaps, thead, (uint4*)d.lst, ctl, (unsigned)cap_chunks, ctl + 1, s);
-  unsigned ctl_h[2] = {0, 0};
-  if (e == cudaSuccess) e = cudaMemcpyAsync(ctl_h, ctl, 8, cudaMemcpyDeviceToHost, s);
+                    tgaps, thead, (uint4*)d.lst, ctl, (unsigned)cap_chunks, ctl + 2, s);
+  unsigned ctl_h[3] = {0, 0, 0};
+  if (e == cudaSuccess) e = cudaMemcpyAsync(ctl_h, ctl, 12, cudaMemcpyDeviceToHost, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return fail(EFFORT_ERR_CUDA);
-  if (ctl_h[1] & kStatusNonfiniteW) return fail(EFFORT_ERR_NONFINITE);
-  if (ctl_h[1] & kStatusInternal) return fail(EFFORT_ERR_DEVICE);
+  if (ctl_h[2] & kStatusNonfiniteW) return fail(EFFORT_ERR_NONFINITE);
+  if (ctl_h[2] & kStatusInternal) return fail(EFFORT_ERR_DEVICE);
+  d.wmax_bits = ctl_h[1];
 
   // the used chunks into storage of the exact size
   const size_t nch = ctl_h[0];

@@ -24,6 +24,7 @@
 //     (dstride = O rounded up to a multiple of 256).
 //   * probes: [I][16] |w| bits at the midpoint ranks of 16 equal segments of
 //     the kept list (the `get_probes` step of the pages' pseudo-code).
+//   * wmax_bits: the largest kept |w| (bounds every partial sum of a call).
 #pragma once
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -37,8 +38,16 @@ constexpr int kStripe = 256;      // dense stripe: 32 lanes x 8 columns
 constexpr int kCS = 64;           // slots per chunk: 8 lanes x 8 slots
 constexpr int kLanesPerChunk = kCS / 8;
 constexpr int kStoreNum = 3, kStoreDen = 8;  // stored share of every list
-constexpr int kThreads = 1024;    // threads of the matvec kernel (one block per SM)
-constexpr int kWarps = kThreads / 32;
+// Matvec kernel: one block per SM, all resident at once; 16 warps, which
+// stream the block's work units with plain 16-byte loads (dense units: warp w
+// owns 256-column stripe w mod 8 of half the units; sparse chunks: 8 lanes per
+// chunk).
+constexpr int kWarps = 16;
+constexpr int kThreads = kWarps * 32;
+constexpr int kUnitCap = kThreads;    // work units of a block handled per round (one per thread)
+constexpr int kChunkCap = 8192;       // sparse chunks of a round (more: the rest are read dense)
+constexpr int kDenseBatch = 8;        // dense units a warp has in flight
+constexpr int kSparseBatch = 8;       // sparse chunks a lane group has in flight
 constexpr int kPrepThreads = 1024;
 constexpr int kDenseThreads = 256;
 constexpr int kDenseRowsPerItem = 8;  // dense rows a warp accumulates per stripe item
@@ -51,7 +60,7 @@ enum : unsigned { kStatusNonfiniteV = 1u, kStatusNonfiniteW = 2u, kStatusInterna
 
 // radix-select digits of the non-negative fp32 chart: bits [30:19], [18:9], [8:0]
 constexpr int kBins0 = 4096, kBins1 = 1024, kBins2 = 512;
-constexpr int kCandCap = 4096;     // crossing-bin candidates resolved in one block
+constexpr int kCandCap = 4096;     // crossing-bin candidates resolved in one block's shared memory
 
 // Device-resident description of a prepared matrix (passed by value).
 struct HandleDesc {
@@ -63,6 +72,7 @@ struct HandleDesc {
   const uint16_t* probes;  // [I][kP]
   int I, O, n, P, dstride;
   unsigned total_chunks;
+  unsigned wmax_bits;      // binary16 bits of the largest kept |w|
   unsigned long long kept_total;
   int pw[kP];              // probe weights (entries each probe stands for)
 };
@@ -78,14 +88,13 @@ struct WsPtrs {
   unsigned* ghist1;           // [kBins1]
   unsigned* ghist2;           // [kBins2]
   uint2* cand;                // [kCandCap] {chart bits, weight}
-  unsigned* info;             // [I][P]: bit 31 dense, bits 0..30 chunks to read
-  unsigned* rowpre;           // [I][P]: work bytes of the owner block's rows before row i
-  unsigned* ctot;             // [nb][P]: work bytes of each owner block's rows
 };
 // header words: status, candidate count, then 64-bit byte counters: the dense
 // and sparse bytes the running call plans to read (words 8..11) and those of
 // the last finished call (words 12..15)
-enum : int { kHdrStatus = 0, kHdrCand = 1, kHdrDone = 2, kHdrBytesRun = 8, kHdrBytesLast = 12, kHdrWords = 64 };
+// (word 3: the running sum of |v| over the blocks, fp32 bits)
+enum : int { kHdrStatus = 0, kHdrCand = 1, kHdrDone = 2, kHdrVsum = 3, kHdrBytesRun = 8, kHdrBytesLast = 12,
+             kHdrWords = 64 };
 
 struct Job {
   HandleDesc hd;
@@ -106,23 +115,34 @@ constexpr int kMarks = 16;
 // Rows of the chart each block of an nb-block grid owns during the cutoff.
 __host__ __device__ inline int rows_per_block(int I, int nb) { return (I + nb - 1) / nb; }
 
-// Dynamic shared memory of the matvec kernel.
-__host__ __device__ inline size_t smem_layout(int I, int nb, size_t* off_chart, size_t* off_hist, size_t* off_cand,
-                                              size_t* off_lists, size_t* off_ctl) {
+// Shared memory of the matvec kernel (byte offsets).
+struct SmemLayout {
+  size_t chart, absv, hist, hist2, cand, ulst, uhead, uv, utau, dlist, cidx, cunit, ctl, total;
+};
+__host__ __device__ inline SmemLayout smem_layout(int I, int nb) {
+  SmemLayout L;
   const size_t rp = (size_t)rows_per_block(I, nb);
-  size_t o = (size_t)kPW * 4;                         // panel accumulator
-  *off_chart = o;
-  o += rp * kP * 4 + rp * 4 + 64;                     // chart bits and |v| of the owned rows
-  o = (o + 15) / 16 * 16;
-  *off_hist = o;
-  o += (size_t)kBins0 * 4;                            // first-digit histogram / later digits
-  *off_cand = o;
-  o += (size_t)kCandCap * 8;                          // gathered candidates
-  *off_lists = o;
-  o += 64 * 1024;                                     // work lists of the block
-  *off_ctl = o;
-  o += (size_t)(128 + kMaxPanels * (nb + 1)) * 4;     // control words and prefix tables
-  return o;
+  size_t o = (size_t)kPW * 4;                         // fixed-point panel accumulator
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o = (o + bytes + 15) / 16 * 16;
+    return at;
+  };
+  L.chart = take(rp * kP * 4);                        // chart bits of the cutoff rows
+  L.absv = take(rp * 4);                              // |v| of the cutoff rows
+  L.hist = take((size_t)kBins0 * 4);                  // first-digit histogram
+  L.hist2 = take((size_t)(kBins1 + kBins2) * 4);      // second- and third-digit histograms
+  L.cand = take((size_t)kCandCap * 8);                // gathered candidates
+  L.ulst = take((size_t)kUnitCap * 16);               // list records of the round's (row, panel) units
+  L.uhead = take((size_t)kUnitCap * 32);              // their first 16 stored chunks' first magnitudes
+  L.uv = take((size_t)kUnitCap * 4);                  // v of the unit's row
+  L.utau = take((size_t)kUnitCap * 4);                // threshold of the unit's row
+  L.dlist = take((size_t)kUnitCap * 2);               // units read dense
+  L.cidx = take((size_t)kChunkCap * 4);               // sparse chunks to read (chunk index)
+  L.cunit = take((size_t)kChunkCap * 2);              // and the unit of each
+  L.ctl = take(256 * 4);                              // control words
+  L.total = o;
+  return L;
 }
 
 }  // namespace effort

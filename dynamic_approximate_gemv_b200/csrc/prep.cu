@@ -36,7 +36,7 @@ struct PrepArgs {
   uint8_t* gaps;         // capacity cap_chunks * kCS
   uint16_t* head;        // capacity cap_chunks
   uint4* lst;            // [I][P]
-  unsigned* chunk_count; // global chunk allocator
+  unsigned* chunk_count; // global chunk allocator; chunk_count[1] receives max |w| bits of the kept weights
   unsigned cap_chunks;
   unsigned* status;
   int prank[kP];         // probe ranks (-1 for empty segments)
@@ -143,6 +143,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1) k_prep_rows(const __grid_cons
     a.wdense[(size_t)i * a.dstride + j] = row[j];
     atomicAdd(&panel_n[j / kPW], 1);
   }
+  if (threadIdx.x == 0) atomicMax(a.chunk_count + 1, 0x7FFFu - (keys[0] >> 16));
   if (threadIdx.x < kP) {
     const int r = a.prank[threadIdx.x];
     a.probes[(size_t)i * kP + threadIdx.x] = (r >= 0) ? (uint16_t)(0x7FFFu - (keys[r] >> 16)) : (uint16_t)0;

@@ -181,10 +181,9 @@ effort_status_t effort_grid_blocks(effort_handle_t h, int32_t* blocks);
  *     GPU (unordered streams, concurrent host threads) race and give wrong
  *     results; order them on one stream.
  *   Returns EFFORT_ERR_UNSUPPORTED when the handle's geometry needs more than
- *     EFFORT_STATIC_SCRATCH_BYTES of scratch (about 60 KiB plus 8 bytes per
- *     row and 2048-column panel: 4096 x 14336 and 14336 x 4096 need about
- *     0.3 MiB; in_dim x out_dim / 2048 may reach about 250,000), and when
- *     the device ordinal is 64 or above.
+ *     EFFORT_STATIC_SCRATCH_BYTES of scratch (every geometry this build
+ *     supports needs the same 55 KiB: histograms, candidates and a header),
+ *     and when the device ordinal is 64 or above.
  *   The array's address is looked up again whenever the device's primary
  *     context has changed (after cudaDeviceReset), never kept across it.
  */

@@ -78,3 +78,32 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(E, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError):
         E.lib()
+
+
+def test_allocation_cap_gives_nomem_before_any_device_call(L, monkeypatch):
+    """With the library's allocation cap below what a matrix needs,
+    effort_prepare returns EFFORT_ERR_NOMEM (3) before it touches CUDA: the
+    pointer below is never dereferenced and no GPU is present."""
+    vp = ctypes.c_void_p
+    h = vp()
+    fake = vp(0x100000)
+    monkeypatch.setenv("EFFORT_ALLOC_CAP_BYTES", "4096")
+    assert L.effort_prepare(fake, 4096, 14336, ctypes.c_float(1.0), None, ctypes.byref(h)) == 3
+    assert h.value is None
+    assert L.effort_prepare(fake, 64, 64, ctypes.c_float(0.5), None, ctypes.byref(h)) == 3
+    # argument errors still come first
+    assert L.effort_prepare(fake, 0, 64, ctypes.c_float(1.0), None, ctypes.byref(h)) == 1
+    held = ctypes.c_uint64(1)
+    assert L.effort_device_bytes_held(ctypes.byref(held)) == 0
+    assert held.value == 0
+
+
+def test_debug_library_exports_the_same_symbols():
+    """The bounds-checking build (kernels compiled with EFFORT_DEBUG) is a
+    drop-in: it exports every entry point the header declares."""
+    from dynamic_approximate_gemv_b200 import build
+    import dynamic_approximate_gemv_b200 as E
+    build.build()
+    D = ctypes.CDLL(E.LIB_DEBUG_PATH)
+    for name in declared_functions():
+        assert hasattr(D, name), name

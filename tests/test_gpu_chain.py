@@ -104,3 +104,39 @@ def test_chain_per_matrix_effort_schedule(E):
     cycle = (0.05, 0.15, 0.25, 0.5, 1.0)
     names = [n for n, _, _ in bench.CHAIN_MATS]
     run_chain(E, lambda layer, name: cycle[(7 * layer + names.index(name)) % len(cycle)])
+
+
+def test_layer0_full_width_teacher_forced(E):
+    """Layer 0 of the full-width decode stack (q, o 4096 x 4096; k, v
+    4096 x 1024; w1, w3 4096 x 14336; w2 14336 x 4096; keep 0.8; effort
+    0.25), every matvec checked against the oracle on the GPU's own input to
+    that step."""
+    sys.path.insert(0, ROOT)
+    import bench
+    dims, keep, effort = (4096, 1024, 14336), 0.8, 0.25
+    mats = {}
+    for m, (name, a, b) in enumerate(bench.CHAIN_MATS):
+        mats[name] = E.PreparedMatrix(torch.from_numpy(inputs.weights(dims[a], dims[b], m)).cuda(), keep)
+
+    def step(name, x):
+        a, b = [(aa, bb) for n, aa, bb in bench.CHAIN_MATS if n == name][0]
+        m = [k for k, (n, _, _) in enumerate(bench.CHAIN_MATS) if n == name][0]
+        prep = O.Prepared(inputs.weights(dims[a], dims[b], m).view(np.uint16), keep)
+        out = checked_gemv(mats[name], prep, x, effort)
+        del prep
+        return out
+
+    try:
+        xn = bench.rms_norm(torch.from_numpy(inputs.vector(dims[0], 9)).cuda())
+        q = step("q", xn)
+        step("k", xn)
+        step("v", xn)
+        o = step("o", bench.rms_norm(q))
+        h = bench.rms_norm(o)
+        a = step("w1", h)
+        b = step("w3", h)
+        y = step("w2", bench.rms_norm(a * b))
+        assert torch.isfinite(y).all()
+    finally:
+        for pm in mats.values():
+            pm.close()
