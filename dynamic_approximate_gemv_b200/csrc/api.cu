@@ -17,8 +17,9 @@ cudaError_t launch_prep(const uint16_t* W, int I, int O, int n, int P, int dstri
                         uint16_t* wdense, uint16_t* probes, uint16_t* vals, uint8_t* gaps, uint16_t* head, uint4* lst,
                         unsigned* chunk_count, unsigned cap_chunks, unsigned* status, cudaStream_t stream);
 unsigned long long prep_chunk_bound_per_row(int O, int n);
-cudaError_t effort_kernel_attributes(size_t smem);
-int effort_blocks_per_sm(size_t smem);
+size_t effort_smem_bytes(int I, int nb);
+cudaError_t effort_kernel_attributes(int I, size_t smem);
+int effort_grid_size(int I, int sms, size_t smem);
 cudaError_t launch_effort(const Job& job, int nb, size_t smem, cudaStream_t stream);
 cudaError_t launch_dense(const uint16_t* W, int I, int O, const void* v, int vdtype, float* out, float* part,
                          unsigned* tilecnt, int T, int S, cudaStream_t stream);
@@ -99,13 +100,14 @@ effort_status_t make_geometry(int64_t I, int64_t O, int n, Geometry* g) {
   g->dstride = (int)((O + kStripe - 1) / kStripe * kStripe);
   g->T = (int)((O + 255) / 256);
   g->nb = sms;
-  g->smem = smem_layout(g->I, g->nb).total;
+  g->smem = effort_smem_bytes(g->I, sms);
   if (g->smem > (size_t)optin) return EFFORT_ERR_UNSUPPORTED;
-  if (effort_kernel_attributes(g->smem) != cudaSuccess) {
+  if (effort_kernel_attributes(g->I, g->smem) != cudaSuccess) {
     cudaGetLastError();
     return EFFORT_ERR_CUDA;
   }
-  if (effort_blocks_per_sm(g->smem) < 1) return EFFORT_ERR_UNSUPPORTED;
+  g->nb = effort_grid_size(g->I, sms, g->smem);  // every block must be resident at once
+  if (g->nb < 1) return EFFORT_ERR_UNSUPPORTED;
   int Sd = (sms * dense_ctas_per_sm()) / g->T;
   if (Sd < 1) Sd = 1;
   if (Sd > (int)((I + 7) / 8)) Sd = (int)((I + 7) / 8);

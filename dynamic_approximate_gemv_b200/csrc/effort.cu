@@ -827,17 +827,30 @@ __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ 
 }
 
 // ------------------------------------------------------------------ launch
-cudaError_t effort_kernel_attributes(size_t smem) {
-  return cudaFuncSetAttribute(k_effort, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+size_t effort_smem_bytes(int I, int nb) { return smem_layout(I, nb).total; }
+
+// The kernel may take up to the device's opt-in shared memory per block: the
+// attribute is a per-function setting, so it must cover every prepared
+// geometry at once (the one a later effort_prepare needs may be smaller).
+cudaError_t effort_kernel_attributes(int I, size_t smem) {
+  (void)I;
+  int dev = 0, optin = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  if (e != cudaSuccess) return e;
+  if ((size_t)optin < smem) return cudaErrorInvalidValue;
+  return cudaFuncSetAttribute(k_effort, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
 }
 
-int effort_blocks_per_sm(size_t smem) {
+// Blocks of a launch that can all be resident at once: one per SM.
+int effort_grid_size(int I, int sms, size_t smem) {
+  (void)I;
   int nbk = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nbk, k_effort, kThreads, smem) != cudaSuccess) {
     cudaGetLastError();
     return 0;
   }
-  return nbk;
+  return nbk >= 1 ? sms : 0;
 }
 
 cudaError_t launch_effort(const Job& job, int nb, size_t smem, cudaStream_t stream) {

@@ -334,6 +334,18 @@ def test_ffn_shapes_full_size(E, I, Od, keep):
     pm.close()
 
 
+def test_handles_of_different_geometries_interleave(E):
+    """Each geometry needs its own amount of shared memory per block; a
+    matrix prepared after another one with a smaller need must not leave the
+    first one unable to launch."""
+    Wb, prep_b, pm_b = make(E, 14336, 1024, 81)   # the larger per-block need
+    Ws, prep_s, pm_s = make(E, 512, 1024, 82)     # prepared afterwards
+    for pm, prep, I in ((pm_b, prep_b, 14336), (pm_s, prep_s, 512), (pm_b, prep_b, 14336)):
+        check_call(E, prep, pm, inputs.vector(I, 83, "t3"), 0.25)
+    pm_b.close()
+    pm_s.close()
+
+
 def test_tie_heavy_input_takes_the_many_candidates_path(E):
     """Constant |v| and W drawn from eight magnitudes give the chart eight
     distinct values, so the crossing bin holds one value shared by about
