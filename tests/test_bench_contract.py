@@ -58,3 +58,18 @@ def test_reference_arm_prints_one_contract_line():
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["sample"] and cb["value"] == d["value"]
     assert d["e2e"] == {"value": d["value"], "unit": "us", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
     assert d["config"]["workload"].startswith("approx GEMV W 4096x14336")
+
+
+def test_byte_counts_per_path():
+    """Algorithmic bytes: 3 per used product, the 16 fp16 probes of every
+    row, v and out; read bytes: what the call plans to read per path (dense
+    panel rows, stored chunks) plus the same probes, v and out.  At effort 1
+    the read figure is the dense copy's 2 bytes per entry, so a bandwidth
+    computed from it cannot exceed a copy's."""
+    import bench
+    I, O = 4096, 14336
+    assert bench.algorithmic_bytes(I, O, 0) == 32 * I + 4 * I + 4 * O
+    assert bench.algorithmic_bytes(I, O, 1000) - bench.algorithmic_bytes(I, O, 0) == 3000
+    assert bench.read_bytes(I, O, 2 * I * O, 0) == 2 * I * O + 32 * I + 4 * I + 4 * O
+    assert bench.read_bytes(I, O, 10, 20, v_bytes=2) == 30 + 32 * I + 2 * I + 4 * O
+    assert bench.read_bytes(I, O, 2 * I * O, 0) < bench.algorithmic_bytes(I, O, I * O)
