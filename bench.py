@@ -807,8 +807,8 @@ def main():
     chain = measure_chain(E, dev) if (not a.no_sweep and world == 1) else {}
 
     # end to end through the C ABI on host buffers (effort_gemv_host): every
-    # step reads its v from pinned host memory (in place, across the host
-    # link) and copies out back to pinned host memory; the library calls are
+    # step copies its v from pinned host memory into the device and copies out
+    # back to pinned host memory; the library calls are
     # issued from a CUDA graph of GRAPH_STEPS calls, like the device-resident
     # steps, so the figure carries the transfers and not Python's call cost
     n_e2e = max(1, min(a.steps, 400) // GRAPH_STEPS) * GRAPH_STEPS
@@ -854,7 +854,7 @@ def main():
                 "e2e": {"value": e2e_us, "unit": "us", "h2d_bytes_per_step": 4 * IN_DIM,
                         "d2h_bytes_per_step": 4 * OUT_DIM,
                         "how": "effort_gemv_host (C ABI) on pinned host v and out, calls issued from CUDA graphs of "
-                               f"{GRAPH_STEPS}; v read in place across the host link, out copied back every step"},
+                               f"{GRAPH_STEPS}; v copied in and out copied back every step"},
                 "gpu_launches": a.steps, "clocks": clocks,
                 "mean_used_products": S_mean, "baselines": baselines, "sweep": sweep,
                 "shapes": shapes,

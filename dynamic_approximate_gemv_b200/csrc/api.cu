@@ -163,17 +163,6 @@ struct DeviceGuard {
 
 }  // namespace
 
-// Device address of page-locked host memory mapped into the device's address
-// space (cudaHostAlloc, cudaMallocHost, cudaHostRegister with mapping), else
-// nullptr (pageable memory, device memory, unknown pointers).
-static void* mapped_host_pointer(const void* p) {
-  cudaPointerAttributes a;
-  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
-    cudaGetLastError();
-    return nullptr;
-  }
-  return (a.type == cudaMemoryTypeHost) ? a.devicePointer : nullptr;
-}
 
 // Offset of out inside effort_gemv_host's staging buffer (v first).
 static size_t stage_out_offset(int I) { return ((size_t)I * 4 + 255) / 256 * 256; }
@@ -429,15 +418,14 @@ effort_status_t effort_gemv_host(effort_handle_t h, const void* v_host, effort_d
   if (!effort_ok(effort)) return EFFORT_ERR_ARG;
   DeviceGuard guard(h->dev);
   cudaStream_t s = (cudaStream_t)stream;
-  // page-locked v mapped into the device's address space is read in place by
-  // the kernel; other host memory is copied into the staging buffer.  out is
-  // accumulated with device-memory reductions, so it always goes through the
-  // staging buffer and one copy back
-  void* mv = mapped_host_pointer(v_host);
-  void* d_v = mv ? mv : h->stage.p;
+  // v is copied into the staging buffer (every block of the kernel reads
+  // it, which in place across the host link would cost a round trip per
+  // block); out is accumulated with device-memory reductions, so it goes
+  // through the staging buffer and one copy back
+  void* d_v = h->stage.p;
   float* d_out = reinterpret_cast<float*>(static_cast<char*>(h->stage.p) + stage_out_offset(h->g.I));
   const size_t vbytes = (size_t)h->g.I * (v_dtype == EFFORT_F16 ? 2 : 4);
-  if (!mv && cudaMemcpyAsync(d_v, v_host, vbytes, cudaMemcpyHostToDevice, s) != cudaSuccess) {
+  if (cudaMemcpyAsync(d_v, v_host, vbytes, cudaMemcpyHostToDevice, s) != cudaSuccess) {
     cudaGetLastError();
     return EFFORT_ERR_CUDA;
   }

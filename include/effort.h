@@ -117,11 +117,10 @@ effort_status_t effort_gemv_ex(effort_handle_t h, const void* v, effort_dtype_t 
  *   library service around the same matvec.  On `stream`, in order, the same
  *   kernel as effort_gemv_ex, with v (in_dim elements of v_dtype) and out
  *   (out_dim fp32) moved across the host link as follows:
- *   - v in page-locked memory mapped into the device's address space
- *     (cudaHostAlloc, cudaMallocHost, cudaHostRegister with mapping;
- *     cudaPointerGetAttributes decides) is read in place by the kernel; other
- *     host memory is copied into the handle's device staging buffer with one
- *     cudaMemcpyAsync before the kernel;
+ *   - v is copied into the handle's device staging buffer with one
+ *     cudaMemcpyAsync before the kernel (every block of the kernel reads v,
+ *     so reading it in place across the host link would cost a host-link
+ *     round trip per block);
  *   - out is accumulated in the staging buffer (the kernel adds partial sums
  *     into it with device-memory reductions) and copied back with one
  *     cudaMemcpyAsync after the kernel.  CUDA stages copies from or to
@@ -143,12 +142,13 @@ effort_status_t effort_gemv_host(effort_handle_t h, const void* v_host, effort_d
  *   timing: marks is a device uint64 array [blocks][16] (blocks from
  *   effort_grid_blocks); entry k of block b is written by that block when it
  *   reaches point k: 0 start, 1 after waiting for the preceding grid, 2 chart
- *   histogram pushed, 3 after the first grid barrier, 4 dispatch bounds
- *   published, 5 after the second grid barrier, 6 cutoff resolved, 7 work
- *   range known, 8 first work lists built, 9 first dense units done, 10 first
- *   round of sparse chunks done, 11 the block's sums added into out, 13 the
- *   block is done (12 is not used).  Points a call does not reach
- *   (effort 1 skips 2..5, a tiny effort returns after 1) keep their old
+ *   histogram pushed, 3 after the first grid barrier, 4 candidates listed,
+ *   5 after the second grid barrier, 6 cutoff resolved, 7 work lists built,
+ *   8 dense units streamed, 9 sparse chunks streamed, 10 registers added into
+ *   the panel accumulator, 11 the block's sums added into out, 13 the block is
+ *   done (12, 14 and 15 are not used); 8 and 9 are written by lane 0 of every
+ *   warp (the last write stays).  Points a call does not reach (effort 1
+ *   skips 2..5, a tiny effort returns after 1) keep their old
  *   contents.  The pages have no counterpart: a measurement service.
  */
 effort_status_t effort_gemv_timed(effort_handle_t h, const void* v, effort_dtype_t v_dtype, float effort,

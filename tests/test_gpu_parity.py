@@ -233,9 +233,8 @@ def test_fp16_vector(E):
 
 @pytest.mark.parametrize("dtype", [np.float32, np.float16])
 def test_host_buffers_match_device_call(E, dtype):
-    """effort_gemv_host (host v in, host out back) gives the device call's
-    output bit for bit, and so the oracle's within the contract, both for
-    pinned buffers (accessed in place) and pageable ones (copied)."""
+    """effort_gemv_host (host v copied in, out copied back) matches the
+    oracle within the contract, for pinned and pageable buffers."""
     _, prep, pm = make(E, 1000, 1300, 21, keep=0.9)
     v_np = inputs.vector(1000, 22, "t3", dtype=dtype)
     v_host = torch.from_numpy(v_np).pin_memory()
@@ -244,13 +243,13 @@ def test_host_buffers_match_device_call(E, dtype):
     torch.cuda.synchronize()
     ref = O.effort_gemv(prep, v_np, 0.3).out
     assert_out_close(out_host.numpy(), ref)
-    # pageable host memory goes through the staging buffer and copies
+    # pageable host memory: the same copies, staged by CUDA
     out2 = torch.zeros(1300, dtype=torch.float32)
     pm.gemv_host(torch.from_numpy(v_np), 0.3, out2)
     torch.cuda.synchronize()
     assert_out_close(out2.numpy(), ref)
-    # pinned buffers are read and written in place: new contents of the same
-    # buffers between calls are seen, call after call
+    # new contents written into the same pinned buffers between calls are
+    # seen, call after call
     for seed in (23, 24, 25):
         w_np = inputs.vector(1000, seed, "normal", dtype=dtype)
         v_host.copy_(torch.from_numpy(w_np))
