@@ -7,6 +7,7 @@
 #include <string.h>
 
 #include <atomic>
+#include <vector>
 #include <new>
 
 #include "../../include/effort.h"
@@ -20,7 +21,7 @@ unsigned long long prep_chunk_bound_per_row(int O, int n);
 size_t effort_smem_bytes(int I, int nb);
 cudaError_t effort_kernel_attributes(int I, size_t smem);
 int effort_grid_size(int I, int sms, size_t smem);
-cudaError_t launch_effort(const Job& job, int nb, size_t smem, cudaStream_t stream);
+cudaError_t launch_effort(const Job& job, int nb, size_t smem, cudaStream_t stream, int nvec = 1);
 cudaError_t launch_dense(const uint16_t* W, int I, int O, const void* v, int vdtype, float* out, float* part,
                          unsigned* tilecnt, int T, int S, cudaStream_t stream);
 int dense_ctas_per_sm();
@@ -187,6 +188,8 @@ struct effort_workspace_s {
   int max_pairs = 0;
   DevBuf ws;
   WsPtrs slot = {};
+  DevBuf ws2;          // the second vector's scratch of a two-vector launch
+  WsPtrs slot2 = {};
   DevBuf dense_part;  // dense baseline: partial tiles and arrival counters
   cudaStream_t last_stream = nullptr;
 };
@@ -477,12 +480,21 @@ effort_status_t effort_workspace_create(int64_t in_dim, int64_t out_dim, int32_t
     w->slot = carve((char*)w->ws.p, w->g);
     if (clear_scratch(w->slot, nullptr) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) st = EFFORT_ERR_CUDA;
   }
+  if (st == EFFORT_OK && max_pairs >= 2) {
+    st = w->ws2.alloc(scratch_bytes(w->g));
+    if (st == EFFORT_OK) {
+      w->slot2 = carve((char*)w->ws2.p, w->g);
+      if (clear_scratch(w->slot2, nullptr) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess)
+        st = EFFORT_ERR_CUDA;
+    }
+  }
   const size_t dense_bytes = align_up((size_t)w->g.S_dense * w->g.T * 256 * 4, 256) + align_up((size_t)w->g.T * 4, 256);
   if (st == EFFORT_OK) st = w->dense_part.alloc(dense_bytes);
   if (st == EFFORT_OK && cudaMemset(w->dense_part.p, 0, dense_bytes) != cudaSuccess) st = EFFORT_ERR_CUDA;
   if (st != EFFORT_OK) {
     cudaGetLastError();
     w->ws.release();
+    w->ws2.release();
     w->dense_part.release();
     delete w;
     return st;
@@ -498,6 +510,7 @@ effort_status_t effort_workspace_destroy(effort_workspace_t w) {
     DeviceGuard guard(w->dev);
     cudaStreamSynchronize(w->last_stream);
     w->ws.release();
+    w->ws2.release();
     w->dense_part.release();
   }
   delete w;
@@ -521,20 +534,63 @@ effort_status_t effort_gemv_batched(effort_workspace_t ws, const effort_handle_t
   DeviceGuard guard(ws->dev);
   cudaStream_t s = (cudaStream_t)stream;
   ws->last_stream = s;
-  // one grid per pair, all on one stream: each grid waits for the one before
-  // it, so the pairs share the workspace's scratch
-  for (int p = 0; p < n_pairs; ++p) {
+  // Pairs on the same matrix whose cutoffs both select go two at a time into
+  // one grid that reads the union of their prefixes once (each keeps its own
+  // cutoff, thresholds and output); the rest run one grid per pair.  All
+  // grids are on one stream, each waiting for the one before, so they share
+  // the workspace's scratch.
+  auto job_of = [&](int p, const WsPtrs& slot, Job* job) {
     effort_handle_t h = handles[hidx[p]];
+    return fill_job(h, slot, (const char*)V + (size_t)vidx[p] * I * vsz, v_dtype, efforts[p], OUT + (size_t)p * O,
+                    cutoffs_out ? cutoffs_out + p : nullptr, counts_out ? counts_out + p : nullptr, nullptr, job);
+  };
+  auto launch_one = [&](int p) -> effort_status_t {
     Job job;
-    effort_status_t st = fill_job(h, ws->slot, (const char*)V + (size_t)vidx[p] * I * vsz, v_dtype, efforts[p],
-                                  OUT + (size_t)p * O, cutoffs_out ? cutoffs_out + p : nullptr,
-                                  counts_out ? counts_out + p : nullptr, nullptr, &job);
+    effort_status_t st = job_of(p, ws->slot, &job);
     if (st != EFFORT_OK) return st;
-    if (launch_effort(job, ws->g.nb, ws->g.smem, s) != cudaSuccess) {
+    if (launch_effort(job, ws->g.nb, ws->g.smem, s, 1) != cudaSuccess) {
+      cudaGetLastError();
+      return EFFORT_ERR_CUDA;
+    }
+    return EFFORT_OK;
+  };
+  std::vector<int> waiting;  // per handle index: a selecting pair without a partner yet, or -1
+  for (int p = 0; p < n_pairs; ++p) {
+    Job a;
+    effort_status_t st = job_of(p, ws->slot, &a);
+    if (st != EFFORT_OK) return st;
+    const int hx = hidx[p];
+    if ((int)waiting.size() <= hx) waiting.resize(hx + 1, -1);
+    if (a.mode != kModeSelect || !ws->ws2.p) {
+      st = launch_one(p);
+      if (st != EFFORT_OK) return st;
+      continue;
+    }
+    if (waiting[hx] < 0) {
+      waiting[hx] = p;
+      continue;
+    }
+    Job first, second;
+    st = job_of(waiting[hx], ws->slot, &first);
+    if (st == EFFORT_OK) st = job_of(p, ws->slot2, &second);
+    if (st != EFFORT_OK) return st;
+    first.v2 = second.v;
+    first.out2 = second.out;
+    first.cutoff_out2 = second.cutoff_out;
+    first.count_out2 = second.count_out;
+    first.ws2 = second.ws;
+    first.K2 = second.K;
+    waiting[hx] = -1;
+    if (launch_effort(first, ws->g.nb, ws->g.smem, s, 2) != cudaSuccess) {
       cudaGetLastError();
       return EFFORT_ERR_CUDA;
     }
   }
+  for (int hx = 0; hx < (int)waiting.size(); ++hx)
+    if (waiting[hx] >= 0) {
+      const effort_status_t st = launch_one(waiting[hx]);
+      if (st != EFFORT_OK) return st;
+    }
   return EFFORT_OK;
 }
 

@@ -246,10 +246,14 @@ __device__ __forceinline__ unsigned chunks_reaching(const HandleDesc& hd, const 
   return m;
 }
 
+// V vectors per launch (1, or 2 on one matrix: the union of their prefixes is
+// read once and each vector's threshold applied to it).  Per-vector state is
+// held in arrays of V.
+template <int V>
 __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ Job jb) {
   extern __shared__ __align__(128) unsigned char smem[];
   const HandleDesc& hd = jb.hd;
-  const WsPtrs& ws = jb.ws;
+  const WsPtrs& ws = jb.ws;  // vector 0's scratch holds the grid barrier and the call's counters
   const int I = hd.I, O = hd.O, P = hd.P;
   const unsigned nb = gridDim.x;
   const unsigned bnb = jb.barrier_nb;
@@ -267,9 +271,31 @@ __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ 
   const unsigned dense_bytes = (unsigned)stripes * (kStripe * 2);
   const int mode = jb.mode;
 
-  const SmemLayout L = smem_layout(I, (int)nb);
+  // per-vector arguments
+  const void* vptr[V];
+  float* outp[V];
+  float* cutp[V];
+  unsigned long long* cntp[V];
+  WsPtrs wsv[V];
+  unsigned long long Kv[V];
+  vptr[0] = jb.v;
+  outp[0] = jb.out;
+  cutp[0] = jb.cutoff_out;
+  cntp[0] = jb.count_out;
+  wsv[0] = jb.ws;
+  Kv[0] = jb.K;
+  if constexpr (V > 1) {
+    vptr[1] = jb.v2;
+    outp[1] = jb.out2;
+    cutp[1] = jb.cutoff_out2;
+    cntp[1] = jb.count_out2;
+    wsv[1] = jb.ws2;
+    Kv[1] = jb.K2;
+  }
+
+  const SmemLayout L = smem_layout(I, (int)nb, V);
   KSmem S;
-  S.iacc = reinterpret_cast<int*>(smem);
+  S.iacc = reinterpret_cast<int*>(smem + L.iacc);
   S.chart = reinterpret_cast<unsigned*>(smem + L.chart);
   S.absv = reinterpret_cast<float*>(smem + L.absv);
   S.hist = reinterpret_cast<unsigned*>(smem + L.hist);
@@ -285,16 +311,17 @@ __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ 
   S.ctl = reinterpret_cast<unsigned*>(smem + L.ctl);
   unsigned* wsum = S.ctl + kCtlWsum;
   unsigned* status = ws.hdr + kHdrStatus;
+  const int chs = nr * kP;  // chart entries of one vector (the chart of vector k at S.chart + k rp kP)
 
   // The next call may start its prologue as soon as SMs free up.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   EFFORT_MARK(0);
 
   // ---- prologue: prepared-matrix data and shared memory only
-  for (int e = tid; e < nr * kP; e += kThreads) S.chart[e] = hd.probes[(size_t)r0 * kP + e];
-  for (int e = tid; e < kBins0; e += kThreads) S.hist[e] = 0u;
+  for (int e = tid; e < chs; e += kThreads) S.chart[e] = hd.probes[(size_t)r0 * kP + e];
+  for (int e = tid; e < V * kBins0; e += kThreads) S.hist[e] = 0u;
   for (int e = tid; e < kBins1 + kBins2; e += kThreads) S.hist2[e] = 0u;
-  for (int e = tid; e < kPW; e += kThreads) S.iacc[e] = 0;
+  for (int e = tid; e < V * kPW; e += kThreads) S.iacc[e] = 0;
   if (tid < 256) S.ctl[tid] = 0u;
   const int nu0 = min(nu, kUnitCap);  // units of the first round
   if (mode == kModeAll) {
@@ -313,7 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ 
 
   const int oc0 = (int)((long long)O * b / nb), oc1 = (int)((long long)O * (b + 1) / nb);  // this block's columns
 
-  // ---- nothing is used: zero outputs, no grid-wide work
+  // ---- nothing is used: zero outputs, no grid-wide work (one vector only)
   if (mode == kModeNone) {
     for (int j = oc0 + tid; j < oc1; j += kThreads) jb.out[j] = 0.0f;
     if (jb.rowlen_out)
@@ -329,46 +356,58 @@ __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ 
   // this block's columns now.  |v| of the cutoff rows (non-finite entries
   // are flagged) and their sum over the grid, which with the largest |w|
   // bounds every partial sum of out; v of the streaming rows.
-  for (int j = oc0 + tid; j < oc1; j += kThreads) jb.out[j] = 0.0f;
-  const float* vf = reinterpret_cast<const float*>(jb.v);
-  const __half* vh = reinterpret_cast<const __half*>(jb.v);
-  for (int u = tid; u < nu0; u += kThreads) {
-    const int i = j0 + u * nbp;
-    S.uv[u] = jb.vdtype ? __half2float(vh[i]) : vf[i];
-  }
-  for (int t0 = 0; t0 < nr; t0 += kThreads) {
-    const int t = t0 + tid;
-    float ax = 0.0f;
-    if (t < nr) {
-      const float x = jb.vdtype ? __half2float(vh[r0 + t]) : vf[r0 + t];
-      if (!isfinite(x)) atomicOr(status, kStatusNonfiniteV);
-      ax = fabsf(x);
-      S.absv[t] = ax;
-      if (jb.rowlen_out) jb.rowlen_out[r0 + t] = (mode == kModeAll) ? (unsigned)hd.n : 0u;
-    }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ax += __shfl_xor_sync(0xFFFFFFFFu, ax, o);
-    if (lane == 0 && ax != 0.0f) atomicAdd(reinterpret_cast<float*>(ws.hdr + kHdrVsum), ax);
+  for (int k = 0; k < V; ++k) {
+    for (int j = oc0 + tid; j < oc1; j += kThreads) outp[k][j] = 0.0f;
+    const float* vf = reinterpret_cast<const float*>(vptr[k]);
+    const __half* vh = reinterpret_cast<const __half*>(vptr[k]);
+    for (int u = tid; u < nu0; u += kThreads) {
+      const int i = j0 + u * nbp;
+      S.uv[k * kUnitCap + u] = jb.vdtype ? __half2float(vh[i]) : vf[i];
+    }
+    for (int t0 = 0; t0 < nr; t0 += kThreads) {
+      const int t = t0 + tid;
+      float ax = 0.0f;
+      if (t < nr) {
+        const float x = jb.vdtype ? __half2float(vh[r0 + t]) : vf[r0 + t];
+        if (!isfinite(x)) atomicOr(status, kStatusNonfiniteV);
+        ax = fabsf(x);
+        S.absv[k * rp + t] = ax;
+        if (k == 0 && jb.rowlen_out) jb.rowlen_out[r0 + t] = (mode == kModeAll) ? (unsigned)hd.n : 0u;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ax += __shfl_xor_sync(0xFFFFFFFFu, ax, o);
+      if (lane == 0 && ax != 0.0f) atomicAdd(reinterpret_cast<float*>(wsv[k].hdr + kHdrVsum), ax);
+    }
   }
   __syncthreads();
 
-  float c = 0.0f;
-  unsigned vsum_bits = 0;
+  float c[V];
+  unsigned vsum_bits[V];
+#pragma unroll
+  for (int k = 0; k < V; ++k) {
+    c[k] = 0.0f;
+    vsum_bits[k] = 0u;
+  }
   if (mode == kModeSelect) {
-    // ---- phase 1: chart and first-digit histogram
-    for (int e = tid; e < nr * kP; e += kThreads) {
-      const int k = e & (kP - 1);
-      const float x = __fmul_rn(S.absv[e >> 4], h2f(S.chart[e]));
-      const unsigned xb = __float_as_uint(x);
-      S.chart[e] = xb;
-      const unsigned w = (unsigned)hd.pw[k];
-      if (w) atomicAdd(&S.hist[xb >> 19], w);
+    // ---- phase 1: charts and first-digit histograms
+    for (int e = tid; e < chs; e += kThreads) {
+      const unsigned w = (unsigned)hd.pw[e & (kP - 1)];
+      const unsigned pb = S.chart[e];  // probe bits, replaced by vector 0's chart
+#pragma unroll
+      for (int k = V - 1; k >= 0; --k) {
+        const unsigned xb = __float_as_uint(__fmul_rn(S.absv[k * rp + (e >> 4)], h2f(pb)));
+        S.chart[k * rp * kP + e] = xb;
+        if (w) atomicAdd(&S.hist[k * kBins0 + (xb >> 19)], w);
+      }
     }
     __syncthreads();
-    for (int e = tid; e < kBins0; e += kThreads) {
-      const unsigned h = S.hist[e];
-      if (h) atomicAdd(&ws.ghist0[e], h);
-    }
+#pragma unroll
+    for (int k = 0; k < V; ++k)
+      for (int e = tid; e < kBins0; e += kThreads) {
+        const unsigned h = S.hist[k * kBins0 + e];
+        if (h) atomicAdd(&wsv[k].ghist0[e], h);
+      }
     EFFORT_MARK(2);
     __syncthreads();
     if (tid == 0) grid_arrive_thread(ws.bar);
@@ -381,32 +420,36 @@ __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ 
     if (!S.ctl[kCtlFlag]) return;
     EFFORT_MARK(3);
 
-    // ---- phase 2: crossing bin, candidates
-    constexpr int kQ0 = kBins0 / kThreads;
-    unsigned h0[kQ0];
-    vsum_bits = __ldcg(ws.hdr + kHdrVsum);
+    // ---- phase 2: crossing bins, candidates
+    unsigned b1[V], K1[V];
 #pragma unroll
-    for (int q = 0; q < kQ0; ++q) h0[q] = __ldcg(&ws.ghist0[tid * kQ0 + q]);
-    block_crossing<kQ0>(h0, (unsigned)jb.K, wsum, S.ctl + kCtlCross);
-    const unsigned b1 = S.ctl[kCtlCross];
-    const unsigned K1 = S.ctl[kCtlCross + 1];
-    const float lo = __uint_as_float(b1 << 19);  // c >= lo
-    for (int e0 = 0; e0 < nr * kP; e0 += kThreads) {
-      const int e = e0 + tid;
-      bool in = false;
-      unsigned xb = 0, w = 0;
-      if (e < nr * kP) {
-        xb = S.chart[e];
-        w = (unsigned)hd.pw[e & (kP - 1)];
-        in = w != 0 && (xb >> 19) == b1;
-      }
-      const unsigned bal = __ballot_sync(0xFFFFFFFFu, in);
-      if (bal) {
-        unsigned basei = 0;
-        if (lane == 0) basei = atomicAdd(ws.hdr + kHdrCand, (unsigned)__popc(bal));
-        basei = __shfl_sync(0xFFFFFFFFu, basei, 0);
-        const unsigned pos = basei + __popc(bal & ((1u << lane) - 1u));
-        if (in && pos < (unsigned)kCandCap) ws.cand[pos] = make_uint2(xb, w);
+    for (int k = 0; k < V; ++k) {
+      constexpr int kQ0 = kBins0 / kThreads;
+      unsigned h0[kQ0];
+      vsum_bits[k] = __ldcg(wsv[k].hdr + kHdrVsum);
+#pragma unroll
+      for (int q = 0; q < kQ0; ++q) h0[q] = __ldcg(&wsv[k].ghist0[tid * kQ0 + q]);
+      block_crossing<kQ0>(h0, (unsigned)Kv[k], wsum, S.ctl + kCtlCross);
+      b1[k] = S.ctl[kCtlCross];
+      K1[k] = S.ctl[kCtlCross + 1];
+      const unsigned* chart = S.chart + k * rp * kP;
+      for (int e0 = 0; e0 < chs; e0 += kThreads) {
+        const int e = e0 + tid;
+        bool in = false;
+        unsigned xb = 0, w = 0;
+        if (e < chs) {
+          xb = chart[e];
+          w = (unsigned)hd.pw[e & (kP - 1)];
+          in = w != 0 && (xb >> 19) == b1[k];
+        }
+        const unsigned bal = __ballot_sync(0xFFFFFFFFu, in);
+        if (bal) {
+          unsigned basei = 0;
+          if (lane == 0) basei = atomicAdd(wsv[k].hdr + kHdrCand, (unsigned)__popc(bal));
+          basei = __shfl_sync(0xFFFFFFFFu, basei, 0);
+          const unsigned pos = basei + __popc(bal & ((1u << lane) - 1u));
+          if (in && pos < (unsigned)kCandCap) wsv[k].cand[pos] = make_uint2(xb, w);
+        }
       }
     }
     EFFORT_MARK(4);
@@ -424,127 +467,151 @@ __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ 
     __syncthreads();
     if (!S.ctl[kCtlFlag]) return;
     EFFORT_MARK(5);
-    // the first-digit histogram is read by nobody any more: clear this block's share
-    for (int e = b * (kBins0 / 4) / (int)nb * 4 + tid, e1 = (b + 1) * (kBins0 / 4) / (int)nb * 4; e < e1; e += kThreads)
-      ws.ghist0[e] = 0u;
+#pragma unroll
+    for (int k = 0; k < V; ++k)
+      // the first-digit histogram is read by nobody any more: clear this block's share
+      for (int e = b * (kBins0 / 4) / (int)nb * 4 + tid, e1 = (b + 1) * (kBins0 / 4) / (int)nb * 4; e < e1;
+           e += kThreads)
+        wsv[k].ghist0[e] = 0u;
 
-    // ---- phase 3: bits [18:0] of c
-    unsigned* h1 = S.hist2;           // [kBins1]
-    unsigned* h2 = S.hist2 + kBins1;  // [kBins2]
-    unsigned b2 = 0, b3 = 0;
-    // the first 2 kThreads candidates are loaded with the count (the common case)
-    const uint2 cA = __ldcg(&ws.cand[tid]), cB = __ldcg(&ws.cand[tid + kThreads]);
-    const unsigned M = __ldcg(ws.hdr + kHdrCand);
-    if (M <= (unsigned)kCandCap) {
-      if ((unsigned)tid < M) S.cand[tid] = cA;
-      if ((unsigned)(tid + kThreads) < M) S.cand[tid + kThreads] = cB;
-      for (unsigned e0 = 2 * kThreads; e0 < M; e0 += 4 * kThreads) {
-        uint2 t4[4];
+    // ---- phase 3: bits [18:0] of each c
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const unsigned e = e0 + k * kThreads + tid;
-          t4[k] = (e < M) ? __ldcg(&ws.cand[e]) : make_uint2(0u, 0u);
+    for (int k = 0; k < V; ++k) {
+      const WsPtrs& w_ = wsv[k];
+      unsigned* h1 = S.hist2;           // [kBins1]
+      unsigned* h2 = S.hist2 + kBins1;  // [kBins2]
+      const unsigned* chart = S.chart + k * rp * kP;
+      unsigned b2 = 0, b3 = 0;
+      if (k > 0) {
+        // the digit histograms of the previous vector start over
+        __syncthreads();
+        for (int e = tid; e < kBins1 + kBins2; e += kThreads) S.hist2[e] = 0u;
+        __syncthreads();
+      }
+      // the first 2 kThreads candidates are loaded with the count (the common case)
+      const uint2 cA = __ldcg(&w_.cand[tid]), cB = __ldcg(&w_.cand[tid + kThreads]);
+      const unsigned M = __ldcg(w_.hdr + kHdrCand);
+      if (M <= (unsigned)kCandCap) {
+        if ((unsigned)tid < M) S.cand[tid] = cA;
+        if ((unsigned)(tid + kThreads) < M) S.cand[tid + kThreads] = cB;
+        for (unsigned e0 = 2 * kThreads; e0 < M; e0 += 4 * kThreads) {
+          uint2 t4[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const unsigned e = e0 + q * kThreads + tid;
+            t4[q] = (e < M) ? __ldcg(&w_.cand[e]) : make_uint2(0u, 0u);
+          }
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const unsigned e = e0 + q * kThreads + tid;
+            if (e < M) S.cand[e] = t4[q];
+          }
         }
+        __syncthreads();
+        for (unsigned e = tid; e < M; e += kThreads) atomicAdd(&h1[(S.cand[e].x >> 9) & (kBins1 - 1)], S.cand[e].y);
+        __syncthreads();
+        {
+          unsigned hq[kBins1 / kThreads];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const unsigned e = e0 + k * kThreads + tid;
-          if (e < M) S.cand[e] = t4[k];
+          for (int q = 0; q < kBins1 / kThreads; ++q) hq[q] = h1[tid * (kBins1 / kThreads) + q];
+          block_crossing<kBins1 / kThreads>(hq, K1[k], wsum, S.ctl + kCtlCross);
         }
-      }
-      __syncthreads();
-      for (unsigned e = tid; e < M; e += kThreads) atomicAdd(&h1[(S.cand[e].x >> 9) & (kBins1 - 1)], S.cand[e].y);
-      __syncthreads();
-      {
-        unsigned hq[kBins1 / kThreads];
+        b2 = S.ctl[kCtlCross];
+        const unsigned K2 = S.ctl[kCtlCross + 1];
+        for (unsigned e = tid; e < M; e += kThreads) {
+          const unsigned xb = S.cand[e].x;
+          if (((xb >> 9) & (kBins1 - 1)) == b2) atomicAdd(&h2[xb & (kBins2 - 1)], S.cand[e].y);
+        }
+        __syncthreads();
+        {
+          unsigned hq[kBins2 / kThreads];
 #pragma unroll
-        for (int q = 0; q < kBins1 / kThreads; ++q) hq[q] = h1[tid * (kBins1 / kThreads) + q];
-        block_crossing<kBins1 / kThreads>(hq, K1, wsum, S.ctl + kCtlCross);
-      }
-      b2 = S.ctl[kCtlCross];
-      const unsigned K2 = S.ctl[kCtlCross + 1];
-      for (unsigned e = tid; e < M; e += kThreads) {
-        const unsigned xb = S.cand[e].x;
-        if (((xb >> 9) & (kBins1 - 1)) == b2) atomicAdd(&h2[xb & (kBins2 - 1)], S.cand[e].y);
-      }
-      __syncthreads();
-      {
-        unsigned hq[kBins2 / kThreads];
+          for (int q = 0; q < kBins2 / kThreads; ++q) hq[q] = h2[tid * (kBins2 / kThreads) + q];
+          block_crossing<kBins2 / kThreads>(hq, K2, wsum, S.ctl + kCtlCross);
+        }
+        b3 = S.ctl[kCtlCross];
+      } else {
+        // too many candidates for one block: two more grid-wide histogram passes
+        for (int e = tid; e < chs; e += kThreads) {
+          const unsigned xb = chart[e], w = (unsigned)hd.pw[e & (kP - 1)];
+          if (w && (xb >> 19) == b1[k]) atomicAdd(&h1[(xb >> 9) & (kBins1 - 1)], w);
+        }
+        __syncthreads();
+        for (int e = tid; e < kBins1; e += kThreads)
+          if (h1[e]) atomicAdd(&w_.ghist1[e], h1[e]);
+        if (!grid_barrier_block(ws.bar, bar_base + (unsigned long long)(++nbar) * bnb, status, &S.ctl[kCtlFlag]))
+          return;
+        {
+          unsigned hq[kBins1 / kThreads];
 #pragma unroll
-        for (int q = 0; q < kBins2 / kThreads; ++q) hq[q] = h2[tid * (kBins2 / kThreads) + q];
-        block_crossing<kBins2 / kThreads>(hq, K2, wsum, S.ctl + kCtlCross);
-      }
-      b3 = S.ctl[kCtlCross];
-    } else {
-      // too many candidates for one block: two more grid-wide histogram passes
-      for (int e = tid; e < nr * kP; e += kThreads) {
-        const unsigned xb = S.chart[e], w = (unsigned)hd.pw[e & (kP - 1)];
-        if (w && (xb >> 19) == b1) atomicAdd(&h1[(xb >> 9) & (kBins1 - 1)], w);
-      }
-      __syncthreads();
-      for (int e = tid; e < kBins1; e += kThreads)
-        if (h1[e]) atomicAdd(&ws.ghist1[e], h1[e]);
-      if (!grid_barrier_block(ws.bar, bar_base + (unsigned long long)(++nbar) * bnb, status, &S.ctl[kCtlFlag])) return;
-      {
-        unsigned hq[kBins1 / kThreads];
+          for (int q = 0; q < kBins1 / kThreads; ++q) hq[q] = __ldcg(&w_.ghist1[tid * (kBins1 / kThreads) + q]);
+          block_crossing<kBins1 / kThreads>(hq, K1[k], wsum, S.ctl + kCtlCross);
+        }
+        b2 = S.ctl[kCtlCross];
+        const unsigned K2 = S.ctl[kCtlCross + 1];
+        for (int e = tid; e < chs; e += kThreads) {
+          const unsigned xb = chart[e], w = (unsigned)hd.pw[e & (kP - 1)];
+          if (w && (xb >> 19) == b1[k] && ((xb >> 9) & (kBins1 - 1)) == b2) atomicAdd(&h2[xb & (kBins2 - 1)], w);
+        }
+        __syncthreads();
+        for (int e = tid; e < kBins2; e += kThreads)
+          if (h2[e]) atomicAdd(&w_.ghist2[e], h2[e]);
+        if (!grid_barrier_block(ws.bar, bar_base + (unsigned long long)(++nbar) * bnb, status, &S.ctl[kCtlFlag]))
+          return;
+        // ghist1 is read by nobody any more
+        if (b == 0)
+          for (int e = tid; e < kBins1; e += kThreads) w_.ghist1[e] = 0u;
+        {
+          unsigned hq[kBins2 / kThreads];
 #pragma unroll
-        for (int q = 0; q < kBins1 / kThreads; ++q) hq[q] = __ldcg(&ws.ghist1[tid * (kBins1 / kThreads) + q]);
-        block_crossing<kBins1 / kThreads>(hq, K1, wsum, S.ctl + kCtlCross);
+          for (int q = 0; q < kBins2 / kThreads; ++q) hq[q] = __ldcg(&w_.ghist2[tid * (kBins2 / kThreads) + q]);
+          block_crossing<kBins2 / kThreads>(hq, K2, wsum, S.ctl + kCtlCross);
+        }
+        b3 = S.ctl[kCtlCross];
       }
-      b2 = S.ctl[kCtlCross];
-      const unsigned K2 = S.ctl[kCtlCross + 1];
-      for (int e = tid; e < nr * kP; e += kThreads) {
-        const unsigned xb = S.chart[e], w = (unsigned)hd.pw[e & (kP - 1)];
-        if (w && (xb >> 19) == b1 && ((xb >> 9) & (kBins1 - 1)) == b2) atomicAdd(&h2[xb & (kBins2 - 1)], w);
-      }
-      __syncthreads();
-      for (int e = tid; e < kBins2; e += kThreads)
-        if (h2[e]) atomicAdd(&ws.ghist2[e], h2[e]);
-      if (!grid_barrier_block(ws.bar, bar_base + (unsigned long long)(++nbar) * bnb, status, &S.ctl[kCtlFlag])) return;
-      // ghist1 is read by nobody any more
-      if (b == 0)
-        for (int e = tid; e < kBins1; e += kThreads) ws.ghist1[e] = 0u;
-      {
-        unsigned hq[kBins2 / kThreads];
-#pragma unroll
-        for (int q = 0; q < kBins2 / kThreads; ++q) hq[q] = __ldcg(&ws.ghist2[tid * (kBins2 / kThreads) + q]);
-        block_crossing<kBins2 / kThreads>(hq, K2, wsum, S.ctl + kCtlCross);
-      }
-      b3 = S.ctl[kCtlCross];
+      c[k] = __uint_as_float((b1[k] << 19) | (b2 << 9) | b3);
+      if (b == 0 && tid == 0 && cutp[k]) *cutp[k] = c[k];
     }
-    c = __uint_as_float((b1 << 19) | (b2 << 9) | b3);
-    if (b == 0 && tid == 0 && jb.cutoff_out) *jb.cutoff_out = c;
     // c = 0: every kept product is used (fillers, pads and dropped weights add +0)
-    if (c == 0.0f && jb.rowlen_out)
+    if (c[0] == 0.0f && jb.rowlen_out)
       for (int t = tid; t < nr; t += kThreads) jb.rowlen_out[r0 + t] = (unsigned)hd.n;
   } else {
     // every (row, panel) is read whole: the cleared out must be complete
     // before any block adds to it
     if (!grid_barrier_block(ws.bar, bar_base + (unsigned long long)(++nbar) * bnb, status, &S.ctl[kCtlFlag])) return;
-    vsum_bits = __ldcg(ws.hdr + kHdrVsum);
+    vsum_bits[0] = __ldcg(ws.hdr + kHdrVsum);
     if (b == 0 && tid == 0 && jb.cutoff_out) *jb.cutoff_out = 0.0f;
   }
   EFFORT_MARK(6);
 
-  // fixed-point unit of the accumulator: 2^-s with every partial sum below
+  // fixed-point unit of each accumulator: 2^-s with every partial sum below
   // 2^30 units (|sum| <= sum |v_i| max |w| < bound / 2)
-  float sc = 1.0f, inv_sc = 1.0f;
-  {
-    const float bound = 2.0f * __uint_as_float(vsum_bits) * h2f(hd.wmax_bits);
+  float sc[V], inv_sc[V];
+  bool count_all[V];
+#pragma unroll
+  for (int k = 0; k < V; ++k) {
+    sc[k] = 1.0f;
+    inv_sc[k] = 1.0f;
+    const float bound = 2.0f * __uint_as_float(vsum_bits[k]) * h2f(hd.wmax_bits);
     if (bound > 0.0f && isfinite(bound)) {
       int ex = 0;
       frexpf(bound, &ex);  // bound < 2^ex
       const int sh = max(-120, min(120, 30 - ex));
-      sc = ldexpf(1.0f, sh);
-      inv_sc = ldexpf(1.0f, -sh);
+      sc[k] = ldexpf(1.0f, sh);
+      inv_sc[k] = ldexpf(1.0f, -sh);
     }
+    count_all[k] = mode == kModeAll || c[k] == 0.0f;
   }
-  const bool count_all = mode == kModeAll || c == 0.0f;
-  const bool want_rowlen = jb.rowlen_out != nullptr && !count_all;
+  const bool want_rowlen = V == 1 && jb.rowlen_out != nullptr && !count_all[0];
 
-  float2 acc[4];
+  float2 acc[V][4];
 #pragma unroll
-  for (int m = 0; m < 4; ++m) acc[m] = make_float2(0.0f, 0.0f);
-  unsigned long long my_count = 0;
+  for (int k = 0; k < V; ++k)
+#pragma unroll
+    for (int m = 0; m < 4; ++m) acc[k][m] = make_float2(0.0f, 0.0f);
+  unsigned long long my_count[V];
+#pragma unroll
+  for (int k = 0; k < V; ++k) my_count[k] = 0;
   unsigned long long planned_dense = 0, planned_sparse = 0;  // thread 0
   const int sj = warp & 7, half = warp >> 3;                 // dense: stripe, units k = half mod 2
   const int g8 = lane >> 3, sl = lane & 7;                   // sparse: lane group, slot octet
@@ -564,39 +631,53 @@ __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ 
                                                                                             : (unsigned short)0;
         }
       }
-      for (int u = tid; u < nuR; u += kThreads) {
-        const int i = j0 + (u0 + u) * nbp;
-        S.uv[u] = jb.vdtype ? __half2float(vh[i]) : vf[i];
+#pragma unroll
+      for (int k = 0; k < V; ++k) {
+        const float* vf = reinterpret_cast<const float*>(vptr[k]);
+        const __half* vh = reinterpret_cast<const __half*>(vptr[k]);
+        for (int u = tid; u < nuR; u += kThreads) {
+          const int i = j0 + (u0 + u) * nbp;
+          S.uv[k * kUnitCap + u] = jb.vdtype ? __half2float(vh[i]) : vf[i];
+        }
       }
-      if (tid == 0) {
-        S.ctl[kCtlExtraDense] = 0u;
-      }
+      if (tid == 0) S.ctl[kCtlExtraDense] = 0u;
       __syncthreads();
     }
-    // ---- dispatch (one unit per thread): the row's threshold tau_i(c), then
-    // the unit is skipped (nothing reaches tau), read dense (the stored part
-    // of its list does not reach tau) or read as the stored chunks whose
-    // first magnitude reaches tau
+    // ---- dispatch (one unit per thread): each vector's threshold tau_i(c),
+    // the smallest fp16 magnitude m with fl32(|v_i| m) >= c; the unit is
+    // skipped (nothing reaches the lowest threshold), read dense (the stored
+    // part of its list does not reach it) or read as the stored chunks whose
+    // first magnitude reaches it: the union of the vectors' prefixes
     const int u = tid;
     unsigned kind = 0, m = 0, first = 0;  // kind: 0 none, 1 dense, 2 sparse
     if (u < nuR) {
-      unsigned tau = 0u;
-      if (count_all) {
+      unsigned tmin = 0x7C00u;
+      bool all = false;
+#pragma unroll
+      for (int k = 0; k < V; ++k) {
+        unsigned tau = 0u;
+        if (count_all[k]) {
+          all = true;
+        } else {
+          tau = tau_of(fabsf(S.uv[k * kUnitCap + u]), c[k]);
+          tmin = min(tmin, tau);
+        }
+        S.utau[k * kUnitCap + u] = tau;
+      }
+      if (all) {
         kind = 1;
       } else {
-        tau = tau_of(fabsf(S.uv[u]), c);
         const uint4 Lr = S.ulst[u];  // {first chunk, stored chunks, tail, kept}
         first = Lr.x;
-        if (Lr.w != 0u && tau < 0x7C00u) {
-          if (Lr.z >= tau && Lr.z != 0u) {
+        if (Lr.w != 0u && tmin < 0x7C00u) {
+          if (Lr.z >= tmin && Lr.z != 0u) {
             kind = 1;
           } else {
-            m = chunks_reaching(hd, Lr, S.uhead + u * 16, tau, status);
+            m = chunks_reaching(hd, Lr, S.uhead + u * 16, tmin, status);
             kind = m ? 2u : 0u;
           }
         }
       }
-      S.utau[u] = tau;
     }
     unsigned tot = 0;
     const unsigned pos = block_prefix_excl((kind == 1 ? (1u << 16) : 0u) | (kind == 2 ? m : 0u), wsum, &tot);
@@ -629,52 +710,101 @@ __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ 
 
     // ---- multiply: dense units, warp (stripe sj, half) takes units k = half,
     // half + 2, ... of the dense list, kDenseBatch loads in flight per lane
+    if constexpr (V == 1) {
+      if (sj < stripes) {
+        const uint16_t* base = hd.wdense + (size_t)p * kPW + sj * kStripe + 8 * lane;
+        for (unsigned k0 = (unsigned)half; k0 < nd; k0 += 2 * kDenseBatch) {
+          uint4 wv[kDenseBatch];
+          unsigned tq[kDenseBatch];
+          float vq[kDenseBatch];
+          int iq[kDenseBatch];
+#pragma unroll
+          for (int q = 0; q < kDenseBatch; ++q) {
+            const unsigned k = k0 + 2 * q;
+            wv[q] = make_uint4(0u, 0u, 0u, 0u);
+            tq[q] = 0x7C00u;
+            vq[q] = 0.0f;
+            iq[q] = 0;
+            if (k < nd) {
+              const unsigned uu = S.dlist[k];
+              const int i = j0 + (u0 + (int)uu) * nbp;
+              wv[q] = __ldcs(reinterpret_cast<const uint4*>(base + (size_t)i * hd.dstride));
+              tq[q] = S.utau[uu];
+              vq[q] = S.uv[uu];
+              iq[q] = i;
+            }
+          }
+#pragma unroll
+          for (int q = 0; q < kDenseBatch; ++q) {
+            const unsigned tau2 = tq[q] | (tq[q] << 16);
+            const float2 v2 = make_float2(vq[q], vq[q]);
+            const unsigned w4[4] = {wv[q].x, wv[q].y, wv[q].z, wv[q].w};
+            unsigned rc = 0;
+#pragma unroll
+            for (int mm = 0; mm < 4; ++mm) {
+              const unsigned msk = ge_mask(w4[mm], tau2);
+              rc += __popc(msk);
+              const unsigned wm = w4[mm] & msk;
+              const float2 wf = __half22float2(*reinterpret_cast<const __half2*>(&wm));
+              acc[0][mm] = __ffma2_rn(v2, wf, acc[0][mm]);
+            }
+            my_count[0] += rc >> 4;
+            if (want_rowlen) {
+              unsigned r = rc >> 4;
+#pragma unroll
+              for (int o = 16; o > 0; o >>= 1) r += __shfl_xor_sync(0xFFFFFFFFu, r, o);
+              if (lane == 0 && r) atomicAdd(&jb.rowlen_out[iq[q]], r);
+            }
+          }
+        }
+      }
+    } else {
+      // two vectors: one load of each unit, each vector's mask and FMA
     if (sj < stripes) {
       const uint16_t* base = hd.wdense + (size_t)p * kPW + sj * kStripe + 8 * lane;
       for (unsigned k0 = (unsigned)half; k0 < nd; k0 += 2 * kDenseBatch) {
         uint4 wv[kDenseBatch];
-        unsigned tq[kDenseBatch];
-        float vq[kDenseBatch];
-        int iq[kDenseBatch];
+        unsigned uq[kDenseBatch];
 #pragma unroll
         for (int q = 0; q < kDenseBatch; ++q) {
           const unsigned k = k0 + 2 * q;
           wv[q] = make_uint4(0u, 0u, 0u, 0u);
-          tq[q] = 0x7C00u;
-          vq[q] = 0.0f;
-          iq[q] = 0;
+          uq[q] = 0xFFFFu;
           if (k < nd) {
-            const unsigned uu = S.dlist[k];
-            const int i = j0 + (u0 + (int)uu) * nbp;
-            wv[q] = __ldcs(reinterpret_cast<const uint4*>(base + (size_t)i * hd.dstride));
-            tq[q] = S.utau[uu];
-            vq[q] = S.uv[uu];
-            iq[q] = i;
+            uq[q] = S.dlist[k];
+            wv[q] = __ldcs(reinterpret_cast<const uint4*>(base + (size_t)(j0 + (u0 + (int)uq[q]) * nbp) * hd.dstride));
           }
         }
 #pragma unroll
         for (int q = 0; q < kDenseBatch; ++q) {
-          const unsigned tau2 = tq[q] | (tq[q] << 16);
-          const float2 v2 = make_float2(vq[q], vq[q]);
+          const bool okq = uq[q] != 0xFFFFu;
           const unsigned w4[4] = {wv[q].x, wv[q].y, wv[q].z, wv[q].w};
-          unsigned rc = 0;
 #pragma unroll
-          for (int mm = 0; mm < 4; ++mm) {
-            const unsigned msk = ge_mask(w4[mm], tau2);
-            rc += __popc(msk);
-            const unsigned wm = w4[mm] & msk;
-            const float2 wf = __half22float2(*reinterpret_cast<const __half2*>(&wm));
-            acc[mm] = __ffma2_rn(v2, wf, acc[mm]);
-          }
-          my_count += rc >> 4;
-          if (want_rowlen) {
-            unsigned r = rc >> 4;
+          for (int k = 0; k < V; ++k) {
+            const unsigned tau = okq ? S.utau[k * kUnitCap + uq[q]] : 0x7C00u;
+            const float vi = okq ? S.uv[k * kUnitCap + uq[q]] : 0.0f;
+            const unsigned tau2 = tau | (tau << 16);
+            const float2 v2 = make_float2(vi, vi);
+            unsigned rc = 0;
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) r += __shfl_xor_sync(0xFFFFFFFFu, r, o);
-            if (lane == 0 && r) atomicAdd(&jb.rowlen_out[iq[q]], r);
+            for (int mm = 0; mm < 4; ++mm) {
+              const unsigned msk = ge_mask(w4[mm], tau2);
+              rc += __popc(msk);
+              const unsigned wm = w4[mm] & msk;
+              const float2 wf = __half22float2(*reinterpret_cast<const __half2*>(&wm));
+              acc[k][mm] = __ffma2_rn(v2, wf, acc[k][mm]);
+            }
+            my_count[k] += rc >> 4;
+            if (want_rowlen) {
+              unsigned r = rc >> 4;
+#pragma unroll
+              for (int o = 16; o > 0; o >>= 1) r += __shfl_xor_sync(0xFFFFFFFFu, r, o);
+              if (lane == 0 && r && okq) atomicAdd(&jb.rowlen_out[j0 + (u0 + (int)uq[q]) * nbp], r);
+            }
           }
         }
       }
+    }
     }
     EFFORT_MARK_LANE0(8);
 
@@ -702,8 +832,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ 
 #pragma unroll
       for (int q = 0; q < kSparseBatch; ++q) {
         const bool ok = uq[q] != 0xFFFFu;
-        const unsigned tau = ok ? S.utau[uq[q]] : 0x7C00u;
-        const float vi = ok ? S.uv[uq[q]] : 0.0f;
         // gaps to columns: inclusive sums inside the lane, exclusive across the 8 lanes
         int cs[8];
         cs[0] = (int)(gg[q].x & 0xFFu);
@@ -722,29 +850,35 @@ __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ 
         }
         const int basecol = ex - cs[7] - 1;
         const unsigned w4[4] = {vv[q].x, vv[q].y, vv[q].z, vv[q].w};
-        const unsigned tau2 = tau | (tau << 16);
-        unsigned rc = 0;
-        if (ok) {
 #pragma unroll
-          for (int mm = 0; mm < 4; ++mm) {
-            const unsigned msk = ge_mask(w4[mm], tau2);
-            const int ca = basecol + cs[2 * mm], cb = basecol + cs[2 * mm + 1];
-            if ((msk & 0xFFFFu) && EFFORT_IN_RANGE((unsigned)ca < (unsigned)kPW, status)) {
-              atomicAdd(&S.iacc[ca], __float2int_rn(__fmul_rn(vi, h2f(w4[mm] & 0xFFFFu)) * sc));
-              ++rc;
-            }
-            if ((msk & 0xFFFF0000u) && EFFORT_IN_RANGE((unsigned)cb < (unsigned)kPW, status)) {
-              atomicAdd(&S.iacc[cb], __float2int_rn(__fmul_rn(vi, h2f(w4[mm] >> 16)) * sc));
-              ++rc;
+        for (int k = 0; k < V; ++k) {
+          const unsigned tau = ok ? S.utau[k * kUnitCap + uq[q]] : 0x7C00u;
+          const float vi = ok ? S.uv[k * kUnitCap + uq[q]] : 0.0f;
+          const unsigned tau2 = tau | (tau << 16);
+          int* iacc = S.iacc + k * kPW;
+          unsigned rc = 0;
+          if (ok) {
+#pragma unroll
+            for (int mm = 0; mm < 4; ++mm) {
+              const unsigned msk = ge_mask(w4[mm], tau2);
+              const int ca = basecol + cs[2 * mm], cb = basecol + cs[2 * mm + 1];
+              if ((msk & 0xFFFFu) && EFFORT_IN_RANGE((unsigned)ca < (unsigned)kPW, status)) {
+                atomicAdd(&iacc[ca], __float2int_rn(__fmul_rn(vi, h2f(w4[mm] & 0xFFFFu)) * sc[k]));
+                ++rc;
+              }
+              if ((msk & 0xFFFF0000u) && EFFORT_IN_RANGE((unsigned)cb < (unsigned)kPW, status)) {
+                atomicAdd(&iacc[cb], __float2int_rn(__fmul_rn(vi, h2f(w4[mm] >> 16)) * sc[k]));
+                ++rc;
+              }
             }
           }
-        }
-        my_count += rc;
-        if (want_rowlen) {
-          unsigned r = rc;
+          my_count[k] += rc;
+          if (want_rowlen) {
+            unsigned r = rc;
 #pragma unroll
-          for (int o = 4; o > 0; o >>= 1) r += __shfl_xor_sync(0xFFFFFFFFu, r, o, 8);
-          if (ok && sl == 0 && r) atomicAdd(&jb.rowlen_out[j0 + (u0 + (int)uq[q]) * nbp], r);
+            for (int o = 4; o > 0; o >>= 1) r += __shfl_xor_sync(0xFFFFFFFFu, r, o, 8);
+            if (ok && sl == 0 && r) atomicAdd(&jb.rowlen_out[j0 + (u0 + (int)uq[q]) * nbp], r);
+          }
         }
       }
     }
@@ -752,49 +886,57 @@ __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ 
     __syncthreads();
   }
 
-  // dense registers into the panel accumulator (fixed point)
+  // dense registers into the panel accumulators (fixed point)
   if (sj < stripes) {
     const int cl = sj * kStripe + 8 * lane;
 #pragma unroll
-    for (int mm = 0; mm < 4; ++mm) {
-      const int qx = __float2int_rn(acc[mm].x * sc), qy = __float2int_rn(acc[mm].y * sc);
-      if (qx) atomicAdd(&S.iacc[cl + 2 * mm], qx);
-      if (qy) atomicAdd(&S.iacc[cl + 2 * mm + 1], qy);
-    }
+    for (int k = 0; k < V; ++k)
+#pragma unroll
+      for (int mm = 0; mm < 4; ++mm) {
+        const int qx = __float2int_rn(acc[k][mm].x * sc[k]), qy = __float2int_rn(acc[k][mm].y * sc[k]);
+        if (qx) atomicAdd(&S.iacc[k * kPW + cl + 2 * mm], qx);
+        if (qy) atomicAdd(&S.iacc[k * kPW + cl + 2 * mm + 1], qy);
+      }
   }
   __syncthreads();
   EFFORT_MARK(10);
 
   // this block's panel sums, added into out (float4 reductions)
   if (nu > 0) {
-    float* dst = jb.out + (size_t)p * kPW;
-    if (((uintptr_t)jb.out & 15u) == 0) {
-      for (int j = tid; j < pwid / 4; j += kThreads) {
-        const int4 q = reinterpret_cast<const int4*>(S.iacc)[j];
-        if (q.x | q.y | q.z | q.w)
-          atomicAdd(reinterpret_cast<float4*>(dst) + j,
-                    make_float4((float)q.x * inv_sc, (float)q.y * inv_sc, (float)q.z * inv_sc, (float)q.w * inv_sc));
+#pragma unroll
+    for (int k = 0; k < V; ++k) {
+      float* dst = outp[k] + (size_t)p * kPW;
+      const int* ia = S.iacc + k * kPW;
+      if (((uintptr_t)outp[k] & 15u) == 0) {
+        for (int j = tid; j < pwid / 4; j += kThreads) {
+          const int4 q = reinterpret_cast<const int4*>(ia)[j];
+          if (q.x | q.y | q.z | q.w)
+            atomicAdd(reinterpret_cast<float4*>(dst) + j,
+                      make_float4((float)q.x * inv_sc[k], (float)q.y * inv_sc[k], (float)q.z * inv_sc[k],
+                                  (float)q.w * inv_sc[k]));
+        }
+        for (int j = pwid / 4 * 4 + tid; j < pwid; j += kThreads)
+          if (ia[j]) atomicAdd(dst + j, (float)ia[j] * inv_sc[k]);
+      } else {
+        for (int j = tid; j < pwid; j += kThreads)
+          if (ia[j]) atomicAdd(dst + j, (float)ia[j] * inv_sc[k]);
       }
-      for (int j = pwid / 4 * 4 + tid; j < pwid; j += kThreads)
-        if (S.iacc[j]) atomicAdd(dst + j, (float)S.iacc[j] * inv_sc);
-    } else {
-      for (int j = tid; j < pwid; j += kThreads)
-        if (S.iacc[j]) atomicAdd(dst + j, (float)S.iacc[j] * inv_sc);
     }
   }
   EFFORT_MARK(11);
 
-  // ---- used count and planned bytes; the last block to finish publishes them
-  {
-    unsigned long long x = my_count;
+  // ---- used counts and planned bytes; the last block to finish publishes them
+#pragma unroll
+  for (int k = 0; k < V; ++k) {
+    unsigned long long x = my_count[k];
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xFFFFFFFFu, x, o);
-    if (lane == 0 && x && !count_all) atomicAdd(ws.count, x);
-    if (tid == 0) {
-      unsigned long long* run = reinterpret_cast<unsigned long long*>(ws.hdr + kHdrBytesRun);
-      if (planned_dense) atomicAdd(run, planned_dense);
-      if (planned_sparse) atomicAdd(run + 1, planned_sparse);
-    }
+    if (lane == 0 && x && !count_all[k]) atomicAdd(wsv[k].count, x);
+  }
+  if (tid == 0) {
+    unsigned long long* run = reinterpret_cast<unsigned long long*>(ws.hdr + kHdrBytesRun);
+    if (planned_dense) atomicAdd(run, planned_dense);
+    if (planned_sparse) atomicAdd(run + 1, planned_sparse);
   }
   __syncthreads();
   if (tid == 0) {
@@ -806,12 +948,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ 
   if (S.ctl[kCtlLast]) {
     __threadfence();
     if (tid == 0) {
-      const unsigned long long cnt = count_all ? hd.kept_total : __ldcg(ws.count);
-      if (jb.count_out) *jb.count_out = cnt;
-      *ws.count = 0ull;
-      ws.hdr[kHdrCand] = 0u;
+#pragma unroll
+      for (int k = 0; k < V; ++k) {
+        const unsigned long long cnt = count_all[k] ? hd.kept_total : __ldcg(wsv[k].count);
+        if (cntp[k]) *cntp[k] = cnt;
+        *wsv[k].count = 0ull;
+        wsv[k].hdr[kHdrCand] = 0u;
+        wsv[k].hdr[kHdrVsum] = 0u;
+      }
       ws.hdr[kHdrDone] = 0u;
-      ws.hdr[kHdrVsum] = 0u;
       unsigned long long* run = reinterpret_cast<unsigned long long*>(ws.hdr + kHdrBytesRun);
       unsigned long long* last = reinterpret_cast<unsigned long long*>(ws.hdr + kHdrBytesLast);
       last[0] = __ldcg(run);
@@ -819,15 +964,17 @@ __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ 
       run[0] = 0ull;
       run[1] = 0ull;
     }
-    // the last digit's histogram of the many-candidates path is read by nobody any more
+    // the last digit's histograms of the many-candidates path are read by nobody any more
     if (mode == kModeSelect)
-      for (int e = tid; e < kBins2; e += kThreads) ws.ghist2[e] = 0u;
+#pragma unroll
+      for (int k = 0; k < V; ++k)
+        for (int e = tid; e < kBins2; e += kThreads) wsv[k].ghist2[e] = 0u;
   }
   EFFORT_MARK(13);
 }
 
 // ------------------------------------------------------------------ launch
-size_t effort_smem_bytes(int I, int nb) { return smem_layout(I, nb).total; }
+size_t effort_smem_bytes(int I, int nb) { return smem_layout(I, nb, 2).total; }  // covers both forms
 
 // The kernel may take up to the device's opt-in shared memory per block: the
 // attribute is a per-function setting, so it must cover every prepared
@@ -839,32 +986,37 @@ cudaError_t effort_kernel_attributes(int I, size_t smem) {
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
   if (e != cudaSuccess) return e;
   if ((size_t)optin < smem) return cudaErrorInvalidValue;
-  return cudaFuncSetAttribute(k_effort, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+  e = cudaFuncSetAttribute(k_effort<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_effort<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+  return e;
 }
 
 // Blocks of a launch that can all be resident at once: one per SM.
 int effort_grid_size(int I, int sms, size_t smem) {
   (void)I;
   int nbk = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nbk, k_effort, kThreads, smem) != cudaSuccess) {
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nbk, k_effort<2>, kThreads, smem) != cudaSuccess) {
     cudaGetLastError();
     return 0;
   }
   return nbk >= 1 ? sms : 0;
 }
 
-cudaError_t launch_effort(const Job& job, int nb, size_t smem, cudaStream_t stream) {
+// One matvec (nvec = 1) or two on one matrix (nvec = 2, job.v2 ...).  smem is
+// the handle's size, which covers the two-vector layout.
+cudaError_t launch_effort(const Job& job, int nb, size_t smem, cudaStream_t stream, int nvec) {
+  (void)smem;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)nb);
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = smem;
+  cfg.dynamicSmemBytes = smem_layout(job.hd.I, nb, nvec).total;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k_effort, job);
+  return nvec == 2 ? cudaLaunchKernelEx(&cfg, k_effort<2>, job) : cudaLaunchKernelEx(&cfg, k_effort<1>, job);
 }
 
 }  // namespace effort

@@ -109,34 +109,45 @@ struct Job {
   int mode;
   int vdtype;  // 0 f32, 1 f16
   unsigned long long* marks;  // nullable: [grid][kMarks] phase times (measurement entry point)
+  // the second vector of a two-vector launch (same matrix, each its own
+  // cutoff; both in select mode; no row lengths): its v, out, reported
+  // cutoff and count, scratch and target count
+  const void* v2;
+  float* out2;
+  float* cutoff_out2;
+  unsigned long long* count_out2;
+  WsPtrs ws2;
+  unsigned long long K2;
 };
 constexpr int kMarks = 16;
 
 // Rows of the chart each block of an nb-block grid owns during the cutoff.
 __host__ __device__ inline int rows_per_block(int I, int nb) { return (I + nb - 1) / nb; }
 
-// Shared memory of the matvec kernel (byte offsets).
+// Shared memory of the matvec kernel (byte offsets) for V vectors per launch
+// (V = 2: two vectors on one matrix read the union of their prefixes once).
 struct SmemLayout {
-  size_t chart, absv, hist, hist2, cand, ulst, uhead, uv, utau, dlist, cidx, cunit, ctl, total;
+  size_t iacc, chart, absv, hist, hist2, cand, ulst, uhead, uv, utau, dlist, cidx, cunit, ctl, total;
 };
-__host__ __device__ inline SmemLayout smem_layout(int I, int nb) {
+__host__ __device__ inline SmemLayout smem_layout(int I, int nb, int V = 1) {
   SmemLayout L;
   const size_t rp = (size_t)rows_per_block(I, nb);
-  size_t o = (size_t)kPW * 4;                         // fixed-point panel accumulator
+  size_t o = 0;
   auto take = [&](size_t bytes) {
     const size_t at = o;
     o = (o + bytes + 15) / 16 * 16;
     return at;
   };
-  L.chart = take(rp * kP * 4);                        // chart bits of the cutoff rows
-  L.absv = take(rp * 4);                              // |v| of the cutoff rows
-  L.hist = take((size_t)kBins0 * 4);                  // first-digit histogram
+  L.iacc = take((size_t)V * kPW * 4);                 // fixed-point panel accumulators
+  L.chart = take((size_t)V * rp * kP * 4);            // chart bits of the cutoff rows
+  L.absv = take((size_t)V * rp * 4);                  // |v| of the cutoff rows
+  L.hist = take((size_t)V * kBins0 * 4);              // first-digit histograms
   L.hist2 = take((size_t)(kBins1 + kBins2) * 4);      // second- and third-digit histograms
   L.cand = take((size_t)kCandCap * 8);                // gathered candidates
   L.ulst = take((size_t)kUnitCap * 16);               // list records of the round's (row, panel) units
   L.uhead = take((size_t)kUnitCap * 32);              // their first 16 stored chunks' first magnitudes
-  L.uv = take((size_t)kUnitCap * 4);                  // v of the unit's row
-  L.utau = take((size_t)kUnitCap * 4);                // threshold of the unit's row
+  L.uv = take((size_t)V * kUnitCap * 4);              // v of the unit's row
+  L.utau = take((size_t)V * kUnitCap * 4);            // threshold of the unit's row
   L.dlist = take((size_t)kUnitCap * 2);               // units read dense
   L.cidx = take((size_t)kChunkCap * 4);               // sparse chunks to read (chunk index)
   L.cunit = take((size_t)kChunkCap * 2);              // and the unit of each

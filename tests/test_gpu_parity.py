@@ -426,6 +426,36 @@ def test_batched_more_pairs_than_one_launch(E):
         assert_out_close(OUT[p].cpu().numpy(), O.effort_gemv(prep, V[p], 0.25).out)
 
 
+def test_batched_union_of_two_vectors_tie_heavy(E):
+    """Two selecting pairs on one matrix run as one grid that reads the union
+    of their prefixes once.  With a tie-heavy matrix (eight magnitudes) and
+    constant |v| each vector's crossing bin holds more candidates than one
+    block resolves, so both cutoffs take the grid-wide histogram passes
+    inside the shared grid; a third pair on the same matrix runs alone."""
+    rng = np.random.default_rng(91)
+    mags = np.array([0.001, 0.002, 0.004, 0.008, 0.016, 0.03, 0.05, 0.07], np.float16)
+    I, Od = 4096, 2048
+    Wn = (mags[rng.integers(0, 8, size=(I, Od))] * rng.choice(np.array([-1, 1], np.float16), size=(I, Od)))
+    Wn = Wn.astype(np.float16)
+    prep = O.Prepared(Wn.view(np.uint16), 1.0)
+    pm = E.PreparedMatrix(torch.from_numpy(Wn).cuda(), 1.0)
+    V = np.stack([rng.choice(np.array([-0.5, 0.5]), size=I).astype(np.float32) for _ in range(2)]
+                 + [inputs.vector(I, 92)])
+    hidx, vidx, eff = [0, 0, 0], [0, 1, 2], [0.25, 0.4, 0.3]
+    ws = E.Workspace(I, Od, max_pairs=3)
+    cut = torch.empty(3, device="cuda")
+    cnt = torch.zeros(3, device="cuda", dtype=torch.int64)
+    OUT = E.gemv_batched(ws, [pm], hidx, vidx, torch.from_numpy(V).cuda(), eff, cutoffs=cut, counts=cnt)
+    torch.cuda.synchronize()
+    for p in range(3):
+        ref = O.effort_gemv(prep, V[vidx[p]], eff[p])
+        assert f32bits(cut[p].item()) == f32bits(ref.c)
+        assert int(cnt[p].item()) == ref.count
+        assert_out_close(OUT[p].cpu().numpy(), ref.out)
+    ws.close()
+    pm.close()
+
+
 def test_batched_moe_full_size_sampled_pairs(E):
     """The batched / MoE workload at full size: 8 experts of 4096 x 14336,
     16 vectors N(0,1) routed top-2 by a seeded N(0,1)/64 gate (ties to the
