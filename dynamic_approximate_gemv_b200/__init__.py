@@ -74,6 +74,7 @@ def lib():
             "effort_destroy": [vp],
             "effort_device_bytes_held": [ctypes.POINTER(ctypes.c_uint64)],
             "effort_last_call_bytes": [vp, ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(ctypes.c_uint64)],
+            "effort_workspace_last_call_bytes": [vp, ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(ctypes.c_uint64)],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -272,6 +273,14 @@ class Workspace:
             _check(lib().effort_workspace_create(self.in_dim, self.out_dim, self.max_pairs, ctypes.byref(h)),
                    "effort_workspace_create")
         self._h = h
+
+    def last_call_bytes(self):
+        """(dense, sparse) bytes the last batched call's grids planned to read,
+        summed over the grids (synchronises the workspace's stream)."""
+        d, sp = ctypes.c_uint64(), ctypes.c_uint64()
+        _check(lib().effort_workspace_last_call_bytes(self._h, ctypes.byref(d), ctypes.byref(sp)),
+               "effort_workspace_last_call_bytes")
+        return d.value, sp.value
 
     def close(self):
         if getattr(self, "_h", None):

@@ -541,9 +541,17 @@ effort_status_t effort_gemv_batched(effort_workspace_t ws, const effort_handle_t
   // the workspace's scratch.
   auto job_of = [&](int p, const WsPtrs& slot, Job* job) {
     effort_handle_t h = handles[hidx[p]];
-    return fill_job(h, slot, (const char*)V + (size_t)vidx[p] * I * vsz, v_dtype, efforts[p], OUT + (size_t)p * O,
-                    cutoffs_out ? cutoffs_out + p : nullptr, counts_out ? counts_out + p : nullptr, nullptr, job);
+    const effort_status_t st =
+        fill_job(h, slot, (const char*)V + (size_t)vidx[p] * I * vsz, v_dtype, efforts[p], OUT + (size_t)p * O,
+                 cutoffs_out ? cutoffs_out + p : nullptr, counts_out ? counts_out + p : nullptr, nullptr, job);
+    job->accumulate_bytes = 1;  // the call's bytes are the sum over its grids
+    return st;
   };
+  // the call's planned bytes start over
+  if (cudaMemsetAsync(ws->slot.hdr + kHdrBytesLast, 0, 16, s) != cudaSuccess) {
+    cudaGetLastError();
+    return EFFORT_ERR_CUDA;
+  }
   auto launch_one = [&](int p) -> effort_status_t {
     Job job;
     effort_status_t st = job_of(p, ws->slot, &job);
@@ -591,6 +599,20 @@ effort_status_t effort_gemv_batched(effort_workspace_t ws, const effort_handle_t
       const effort_status_t st = launch_one(waiting[hx]);
       if (st != EFFORT_OK) return st;
     }
+  return EFFORT_OK;
+}
+
+effort_status_t effort_workspace_last_call_bytes(effort_workspace_t ws, uint64_t* dense_bytes, uint64_t* sparse_bytes) {
+  if (!ws || !dense_bytes || !sparse_bytes) return EFFORT_ERR_ARG;
+  DeviceGuard guard(ws->dev);
+  unsigned long long b[2] = {0, 0};
+  if (cudaStreamSynchronize(ws->last_stream) != cudaSuccess ||
+      cudaMemcpy(b, ws->slot.hdr + kHdrBytesLast, 16, cudaMemcpyDeviceToHost) != cudaSuccess) {
+    cudaGetLastError();
+    return EFFORT_ERR_CUDA;
+  }
+  *dense_bytes = b[0];
+  *sparse_bytes = b[1];
   return EFFORT_OK;
 }
 

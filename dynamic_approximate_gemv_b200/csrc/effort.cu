@@ -959,8 +959,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ 
       ws.hdr[kHdrDone] = 0u;
       unsigned long long* run = reinterpret_cast<unsigned long long*>(ws.hdr + kHdrBytesRun);
       unsigned long long* last = reinterpret_cast<unsigned long long*>(ws.hdr + kHdrBytesLast);
-      last[0] = __ldcg(run);
-      last[1] = __ldcg(run + 1);
+      last[0] = (jb.accumulate_bytes ? __ldcg(last) : 0ull) + __ldcg(run);
+      last[1] = (jb.accumulate_bytes ? __ldcg(last + 1) : 0ull) + __ldcg(run + 1);
       run[0] = 0ull;
       run[1] = 0ull;
     }

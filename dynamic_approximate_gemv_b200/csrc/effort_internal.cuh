@@ -118,6 +118,7 @@ struct Job {
   unsigned long long* count_out2;
   WsPtrs ws2;
   unsigned long long K2;
+  int accumulate_bytes;  // 1: add the planned bytes to the last-call words (a batched call's launches)
 };
 constexpr int kMarks = 16;
 

@@ -221,8 +221,15 @@ effort_status_t effort_workspace_destroy(effort_workspace_t ws);
  *   HOST arrays of n_pairs entries.  All handles must share in_dim/out_dim
  *   with the workspace.  cutoffs_out [n_pairs] float and counts_out
  *   [n_pairs] uint64 are nullable device arrays.  One cutoff per pair.
- *   Launches one kernel per pair, in order on `stream`; the pairs share the
- *   workspace's scratch.  n_pairs <= the workspace's max_pairs.
+ *   Two pairs on the same handle whose cutoffs both select (0 < K < the kept
+ *   count) run as one kernel that reads the union of their prefixes once:
+ *   each (row, panel) of the matrix is read as far as the lower of the two
+ *   thresholds needs, and each vector's own threshold is applied to it, so
+ *   each pair's cutoff, count and output are those of its own call (outputs
+ *   to rounding).  Every other pair runs as one kernel of its own.  All
+ *   kernels run in order on `stream` and share the workspace's scratch (two
+ *   slots, the second allocated when max_pairs >= 2).  n_pairs <= the
+ *   workspace's max_pairs.
  */
 effort_status_t effort_gemv_batched(effort_workspace_t ws, const effort_handle_t* handles, const int32_t* hidx,
                                     const int32_t* vidx, int32_t n_pairs, const void* V, effort_dtype_t v_dtype,
@@ -289,6 +296,16 @@ effort_status_t effort_destroy(effort_handle_t h);
  *   pointers, non-NULL.
  */
 effort_status_t effort_last_call_bytes(effort_handle_t h, uint64_t* dense_bytes, uint64_t* sparse_bytes);
+
+/*
+ * effort_workspace_last_call_bytes -- the same for the workspace's last
+ *   effort_gemv_batched call: the bytes its grids planned to read, summed
+ *   over the grids (a grid serving two pairs on one matrix reads the union of
+ *   their prefixes once, and counts it once).  Synchronises the workspace's
+ *   last stream.  A measurement service.
+ */
+effort_status_t effort_workspace_last_call_bytes(effort_workspace_t ws, uint64_t* dense_bytes,
+                                                 uint64_t* sparse_bytes);
 
 /* Device memory the library holds at this moment, over all handles and
  * workspaces of the process (the figure EFFORT_ALLOC_CAP_BYTES is checked

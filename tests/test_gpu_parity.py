@@ -456,6 +456,26 @@ def test_batched_union_of_two_vectors_tie_heavy(E):
     pm.close()
 
 
+def test_batched_union_reads_fewer_bytes_than_separate_calls(E):
+    """A two-pair grid on one matrix reads each unit once, as far as the
+    lower threshold needs: its bytes are at least those of either pair alone
+    and at most their sum."""
+    Wn, prep, pm = make(E, 2048, 6000, 95)
+    V = np.stack([inputs.vector(2048, 96, "t3"), inputs.vector(2048, 97, "t3")])
+    Vt = torch.from_numpy(V).cuda()
+    ws = E.Workspace(2048, 6000, max_pairs=2)
+    E.gemv_batched(ws, [pm], [0, 0], [0, 1], Vt, [0.25, 0.15])
+    union = sum(ws.last_call_bytes())
+    alone = []
+    for k, e in enumerate((0.25, 0.15)):
+        pm.gemv(Vt[k], e)
+        alone.append(sum(pm.last_call_bytes()))
+    assert max(alone) <= union <= sum(alone)
+    assert union < sum(alone)
+    ws.close()
+    pm.close()
+
+
 def test_batched_moe_full_size_sampled_pairs(E):
     """The batched / MoE workload at full size: 8 experts of 4096 x 14336,
     16 vectors N(0,1) routed top-2 by a seeded N(0,1)/64 gate (ties to the
