@@ -432,9 +432,24 @@ effort_status_t effort_gemv_host(effort_handle_t h, const void* v_host, effort_d
     cudaGetLastError();
     return EFFORT_ERR_CUDA;
   }
-  const effort_status_t st = effort_gemv_ex(h, d_v, v_dtype, effort, d_out, nullptr, nullptr, nullptr, stream);
+  // page-locked out mapped into the device's address space is written by the
+  // kernel's last block; other host memory is copied back after the kernel
+  void* mout = nullptr;
+  {
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, out_host) == cudaSuccess && a.type == cudaMemoryTypeHost) mout = a.devicePointer;
+    cudaGetLastError();
+  }
+  Job job;
+  effort_status_t st = fill_job(h, h->slot, d_v, v_dtype, effort, d_out, nullptr, nullptr, nullptr, &job);
   if (st != EFFORT_OK) return st;
-  if (cudaMemcpyAsync(out_host, d_out, (size_t)h->g.O * 4, cudaMemcpyDeviceToHost, s) != cudaSuccess) {
+  job.out_mirror = (float*)mout;
+  h->last_stream = s;
+  if (launch_effort(job, h->g.nb, h->g.smem, s) != cudaSuccess) {
+    cudaGetLastError();
+    return EFFORT_ERR_CUDA;
+  }
+  if (!mout && cudaMemcpyAsync(out_host, d_out, (size_t)h->g.O * 4, cudaMemcpyDeviceToHost, s) != cudaSuccess) {
     cudaGetLastError();
     return EFFORT_ERR_CUDA;
   }

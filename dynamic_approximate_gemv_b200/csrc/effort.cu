@@ -342,7 +342,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ 
 
   // ---- nothing is used: zero outputs, no grid-wide work (one vector only)
   if (mode == kModeNone) {
-    for (int j = oc0 + tid; j < oc1; j += kThreads) jb.out[j] = 0.0f;
+    for (int j = oc0 + tid; j < oc1; j += kThreads) {
+      jb.out[j] = 0.0f;
+      if (jb.out_mirror) jb.out_mirror[j] = 0.0f;
+    }
     if (jb.rowlen_out)
       for (int i = r0 + tid; i < r1; i += kThreads) jb.rowlen_out[i] = 0u;
     if (b == 0 && tid == 0) {
@@ -969,6 +972,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ 
 #pragma unroll
       for (int k = 0; k < V; ++k)
         for (int e = tid; e < kBins2; e += kThreads) wsv[k].ghist2[e] = 0u;
+    // every block has added its sums: the finished out to host memory
+    if (jb.out_mirror)
+      for (int j = tid; j < O; j += kThreads) jb.out_mirror[j] = __ldcg(jb.out + j);
   }
   EFFORT_MARK(13);
 }

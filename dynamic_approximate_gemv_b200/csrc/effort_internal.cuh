@@ -119,6 +119,8 @@ struct Job {
   WsPtrs ws2;
   unsigned long long K2;
   int accumulate_bytes;  // 1: add the planned bytes to the last-call words (a batched call's launches)
+  float* out_mirror;     // nullable: page-locked host memory mapped for the device; the finished out is
+                         // written there by the last block (host-buffer entry point)
 };
 constexpr int kMarks = 16;
 

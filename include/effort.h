@@ -122,9 +122,12 @@ effort_status_t effort_gemv_ex(effort_handle_t h, const void* v, effort_dtype_t 
  *     so reading it in place across the host link would cost a host-link
  *     round trip per block);
  *   - out is accumulated in the staging buffer (the kernel adds partial sums
- *     into it with device-memory reductions) and copied back with one
- *     cudaMemcpyAsync after the kernel.  CUDA stages copies from or to
- *     pageable memory, which may block the host.
+ *     into it with device-memory reductions).  When out_host is page-locked
+ *     memory mapped into the device's address space (cudaHostAlloc,
+ *     cudaMallocHost, cudaHostRegister with mapping; cudaPointerGetAttributes
+ *     decides), the kernel's last block writes the finished out into it;
+ *     otherwise it is copied back with one cudaMemcpyAsync after the kernel
+ *     (CUDA stages copies to pageable memory, which may block the host).
  *   v_host, out_host: host memory, non-NULL.
  *   The call does not synchronise: out_host holds the result once the stream
  *   has passed this call (cudaStreamSynchronize, an event).  The caller must

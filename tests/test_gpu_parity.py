@@ -248,6 +248,10 @@ def test_host_buffers_match_device_call(E, dtype):
     pm.gemv_host(torch.from_numpy(v_np), 0.3, out2)
     torch.cuda.synchronize()
     assert_out_close(out2.numpy(), ref)
+    # an effort that targets no product: out is all zeros
+    pm.gemv_host(v_host, 1e-9, out_host)
+    torch.cuda.synchronize()
+    assert not out_host.any()
     # new contents written into the same pinned buffers between calls are
     # seen, call after call
     for seed in (23, 24, 25):
