@@ -75,6 +75,7 @@ def lib():
             "effort_device_bytes_held": [ctypes.POINTER(ctypes.c_uint64)],
             "effort_last_call_bytes": [vp, ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(ctypes.c_uint64)],
             "effort_workspace_last_call_bytes": [vp, ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(ctypes.c_uint64)],
+            "effort_workspace_check": [vp],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -273,6 +274,9 @@ class Workspace:
             _check(lib().effort_workspace_create(self.in_dim, self.out_dim, self.max_pairs, ctypes.byref(h)),
                    "effort_workspace_create")
         self._h = h
+
+    def check(self):
+        _check(lib().effort_workspace_check(self._h), "effort_workspace_check")
 
     def last_call_bytes(self):
         """(dense, sparse) bytes the last batched call's grids planned to read,

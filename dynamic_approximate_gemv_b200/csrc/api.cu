@@ -617,6 +617,23 @@ effort_status_t effort_gemv_batched(effort_workspace_t ws, const effort_handle_t
   return EFFORT_OK;
 }
 
+effort_status_t effort_workspace_check(effort_workspace_t ws) {
+  if (!ws) return EFFORT_ERR_ARG;
+  DeviceGuard guard(ws->dev);
+  unsigned int st = 0;
+  if (cudaStreamSynchronize(ws->last_stream) != cudaSuccess) return EFFORT_ERR_CUDA;
+  if (cudaMemcpy(&st, ws->slot.hdr + kHdrStatus, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return EFFORT_ERR_CUDA;
+  if (st) {
+    // a timed-out grid leaves the scratch mid-call: start both slots over
+    if (clear_scratch(ws->slot, ws->last_stream) != cudaSuccess) return EFFORT_ERR_CUDA;
+    if (ws->ws2.p && clear_scratch(ws->slot2, ws->last_stream) != cudaSuccess) return EFFORT_ERR_CUDA;
+    if (cudaStreamSynchronize(ws->last_stream) != cudaSuccess) return EFFORT_ERR_CUDA;
+  }
+  if (st & (kStatusInternal | kStatusTimeout)) return EFFORT_ERR_DEVICE;
+  if (st & kStatusNonfiniteV) return EFFORT_ERR_NONFINITE;
+  return EFFORT_OK;
+}
+
 effort_status_t effort_workspace_last_call_bytes(effort_workspace_t ws, uint64_t* dense_bytes, uint64_t* sparse_bytes) {
   if (!ws || !dense_bytes || !sparse_bytes) return EFFORT_ERR_ARG;
   DeviceGuard guard(ws->dev);

@@ -301,6 +301,15 @@ effort_status_t effort_destroy(effort_handle_t h);
 effort_status_t effort_last_call_bytes(effort_handle_t h, uint64_t* dense_bytes, uint64_t* sparse_bytes);
 
 /*
+ * effort_workspace_check -- effort_check for the workspace's calls
+ *   (effort_gemv_batched, effort_dense_gemv): synchronises its last stream,
+ *   reports EFFORT_ERR_NONFINITE if a pair's v held inf or NaN and
+ *   EFFORT_ERR_DEVICE after a timed-out wait or an out-of-range index (debug
+ *   build), clears the flags and, after an error, the workspace's scratch.
+ */
+effort_status_t effort_workspace_check(effort_workspace_t ws);
+
+/*
  * effort_workspace_last_call_bytes -- the same for the workspace's last
  *   effort_gemv_batched call: the bytes its grids planned to read, summed
  *   over the grids (a grid serving two pairs on one matrix reads the union of

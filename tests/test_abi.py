@@ -70,6 +70,7 @@ def test_argument_errors_need_no_device(L):
     assert L.effort_dense_gemv(None, fake, 4, 4, fake, 0, fake, None) == 1
     assert L.effort_get_info(None, None, None, None, None) == 1
     assert L.effort_get_layout(None, None) == 1
+    assert L.effort_workspace_check(None) == 1
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):

@@ -460,6 +460,27 @@ def test_batched_union_of_two_vectors_tie_heavy(E):
     pm.close()
 
 
+def test_batched_nonfinite_vector_is_reported(E):
+    """A non-finite entry in one pair's v of a batched call (here inside a
+    two-pair grid) is reported by the workspace's check, which then clears."""
+    Wn, prep, pm = make(E, 256, 1024, 98)
+    V = np.stack([inputs.vector(256, 99), inputs.vector(256, 100)])
+    V[1, 17] = np.inf
+    ws = E.Workspace(256, 1024, max_pairs=2)
+    E.gemv_batched(ws, [pm], [0, 0], [0, 1], torch.from_numpy(V).cuda(), [0.25, 0.25])
+    with pytest.raises(E.EffortError) as ei:
+        ws.check()
+    assert ei.value.status == 4
+    ws.check()
+    V[1, 17] = 0.5
+    OUT = E.gemv_batched(ws, [pm], [0, 0], [0, 1], torch.from_numpy(V).cuda(), [0.25, 0.25])
+    ws.check()
+    for k in range(2):
+        assert_out_close(OUT[k].cpu().numpy(), O.effort_gemv(prep, V[k], 0.25).out)
+    ws.close()
+    pm.close()
+
+
 def test_batched_union_reads_fewer_bytes_than_separate_calls(E):
     """A two-pair grid on one matrix reads each unit once, as far as the
     lower threshold needs: its bytes are at least those of either pair alone
