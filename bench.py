@@ -675,8 +675,8 @@ def main():
             m = marks.cpu().numpy().astype(np.int64)
             rows.append(m - m[:, 1].min())
         R = np.stack(rows)
-        names = {0: "start", 1: "wait", 2: "chart_histogram", 3: "barrier_B1", 4: "candidates", 5: "barrier_B2",
-                 6: "cutoff", 7: "dispatch", 8: "dense_streamed", 9: "sparse_streamed", 10: "accumulated",
+        names = {0: "start", 1: "wait", 2: "chart_histogram", 3: "barrier_B1", 4: "crossing_bin",
+                 5: "crossing_entries", 6: "cutoff", 7: "dispatch", 8: "dense_streamed", 9: "sparse_streamed", 10: "accumulated",
                  11: "out_reduced", 13: "end"}
         res = {}
         for k, nm in names.items():

@@ -108,7 +108,8 @@ effort_status_t make_geometry(int64_t I, int64_t O, int n, Geometry* g) {
     return EFFORT_ERR_CUDA;
   }
   g->nb = effort_grid_size(g->I, sms, g->smem);  // every block must be resident at once
-  if (g->nb < 1) return EFFORT_ERR_UNSUPPORTED;
+  if (g->nb < 1 || g->nb > kMaxGrid || (long long)rows_per_block(g->I, g->nb) * kP > kMaxSegEntries)
+    return EFFORT_ERR_UNSUPPORTED;
   int Sd = (sms * dense_ctas_per_sm()) / g->T;
   if (Sd < 1) Sd = 1;
   if (Sd > (int)((I + 7) / 8)) Sd = (int)((I + 7) / 8);
@@ -118,15 +119,19 @@ effort_status_t make_geometry(int64_t I, int64_t O, int n, Geometry* g) {
 
 // ---------------------------------------------------------------- scratch
 // Bytes of one call's scratch, carved in this order.
+static size_t desc_bytes(const Geometry& g) { return (size_t)kBins0 * g.nb * 4; }
+static size_t seg_bytes(const Geometry& g) { return (size_t)g.nb * rows_per_block(g.I, g.nb) * kP * 8; }
 size_t scratch_bytes(const Geometry& g) {
   return align_up((size_t)kHdrWords * 4 + 16, 256)                 // header, barrier, count
          + align_up((size_t)(kBins0 + kBins1 + kBins2) * 4, 256)   // histograms
-         + align_up((size_t)kCandCap * 8, 256)                     // candidates
+         + align_up(desc_bytes(g), 256)                            // first-digit bin descriptors
+         + align_up(seg_bytes(g), 256)                             // chart entries grouped by bin
          ;
 }
-// Bytes that must be zero before the first call (header and histograms).
-size_t scratch_zero_bytes() {
-  return align_up((size_t)kHdrWords * 4 + 16, 256) + align_up((size_t)(kBins0 + kBins1 + kBins2) * 4, 256);
+// Bytes that must be zero before the first call (header, histograms, descriptors).
+size_t scratch_zero_bytes(const Geometry& g) {
+  return align_up((size_t)kHdrWords * 4 + 16, 256) + align_up((size_t)(kBins0 + kBins1 + kBins2) * 4, 256) +
+         align_up(desc_bytes(g), 256);
 }
 
 WsPtrs carve(char* b, const Geometry& g) {
@@ -139,8 +144,9 @@ WsPtrs carve(char* b, const Geometry& g) {
   w.ghist1 = w.ghist0 + kBins0;
   w.ghist2 = w.ghist1 + kBins1;
   b += align_up((size_t)(kBins0 + kBins1 + kBins2) * 4, 256);
-  w.cand = (uint2*)b;
-  (void)g;
+  w.desc = (unsigned*)b;
+  b += align_up(desc_bytes(g), 256);
+  w.seg = (uint2*)b;
   return w;
 }
 
@@ -196,16 +202,15 @@ struct effort_workspace_s {
 
 namespace effort {
 
-// The scratch header words, barrier counter and histograms start at zero.
-cudaError_t clear_scratch(const WsPtrs& w, cudaStream_t s) {
-  cudaError_t e = cudaMemsetAsync(w.hdr, 0, align_up((size_t)kHdrWords * 4 + 16, 256), s);
-  if (e == cudaSuccess) e = cudaMemsetAsync(w.ghist0, 0, (size_t)(kBins0 + kBins1 + kBins2) * 4, s);
-  return e;
+// The scratch header words, barrier counter, histograms and bin descriptors
+// start at zero (they are contiguous from the header).
+cudaError_t clear_scratch(const WsPtrs& w, const Geometry& g, cudaStream_t s) {
+  return cudaMemsetAsync(w.hdr, 0, scratch_zero_bytes(g), s);
 }
 
 size_t handle_scratch_bytes(effort_handle_t h) { return scratch_bytes(h->g); }
 WsPtrs handle_carve(effort_handle_t h, char* base) { return carve(base, h->g); }
-size_t handle_scratch_zero_bytes() { return scratch_zero_bytes(); }
+size_t handle_scratch_zero_bytes(effort_handle_t h) { return scratch_zero_bytes(h->g); }
 
 static effort_status_t fill_job(effort_handle_t h, const WsPtrs& ws, const void* v, effort_dtype_t v_dtype,
                                 float effort, float* out, float* cutoff_out, uint64_t* count_out,
@@ -369,7 +374,7 @@ effort_status_t effort_prepare(const void* W, int64_t in_dim, int64_t out_dim, f
   // per-call scratch and the host-call staging buffer
   if ((st = h->ws.alloc(scratch_bytes(h->g))) != EFFORT_OK) return fail(st);
   h->slot = carve((char*)h->ws.p, h->g);
-  if (clear_scratch(h->slot, s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess) return fail(EFFORT_ERR_CUDA);
+  if (clear_scratch(h->slot, h->g, s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess) return fail(EFFORT_ERR_CUDA);
   if ((st = h->stage.alloc(stage_out_offset(I) + (size_t)O * 4)) != EFFORT_OK) return fail(st);
   *out_handle = h;
   return EFFORT_OK;
@@ -469,7 +474,7 @@ effort_status_t effort_check(effort_handle_t h) {
   if (st) {
     // a timed-out grid leaves the barrier counter and histograms mid-call:
     // start the scratch over (the status word with it)
-    if (clear_scratch(h->slot, h->last_stream) != cudaSuccess || cudaStreamSynchronize(h->last_stream) != cudaSuccess)
+    if (clear_scratch(h->slot, h->g, h->last_stream) != cudaSuccess || cudaStreamSynchronize(h->last_stream) != cudaSuccess)
       return EFFORT_ERR_CUDA;
   }
   if (st & (kStatusInternal | kStatusTimeout)) return EFFORT_ERR_DEVICE;
@@ -493,13 +498,13 @@ effort_status_t effort_workspace_create(int64_t in_dim, int64_t out_dim, int32_t
   if (st == EFFORT_OK) st = w->ws.alloc(scratch_bytes(w->g));
   if (st == EFFORT_OK) {
     w->slot = carve((char*)w->ws.p, w->g);
-    if (clear_scratch(w->slot, nullptr) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) st = EFFORT_ERR_CUDA;
+    if (clear_scratch(w->slot, w->g, nullptr) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) st = EFFORT_ERR_CUDA;
   }
   if (st == EFFORT_OK && max_pairs >= 2) {
     st = w->ws2.alloc(scratch_bytes(w->g));
     if (st == EFFORT_OK) {
       w->slot2 = carve((char*)w->ws2.p, w->g);
-      if (clear_scratch(w->slot2, nullptr) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess)
+      if (clear_scratch(w->slot2, w->g, nullptr) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess)
         st = EFFORT_ERR_CUDA;
     }
   }
@@ -625,8 +630,8 @@ effort_status_t effort_workspace_check(effort_workspace_t ws) {
   if (cudaMemcpy(&st, ws->slot.hdr + kHdrStatus, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return EFFORT_ERR_CUDA;
   if (st) {
     // a timed-out grid leaves the scratch mid-call: start both slots over
-    if (clear_scratch(ws->slot, ws->last_stream) != cudaSuccess) return EFFORT_ERR_CUDA;
-    if (ws->ws2.p && clear_scratch(ws->slot2, ws->last_stream) != cudaSuccess) return EFFORT_ERR_CUDA;
+    if (clear_scratch(ws->slot, ws->g, ws->last_stream) != cudaSuccess) return EFFORT_ERR_CUDA;
+    if (ws->ws2.p && clear_scratch(ws->slot2, ws->g, ws->last_stream) != cudaSuccess) return EFFORT_ERR_CUDA;
     if (cudaStreamSynchronize(ws->last_stream) != cudaSuccess) return EFFORT_ERR_CUDA;
   }
   if (st & (kStatusInternal | kStatusTimeout)) return EFFORT_ERR_DEVICE;

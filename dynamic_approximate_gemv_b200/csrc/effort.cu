@@ -14,17 +14,20 @@
 //   x_ik = fl32(|v_i| p_ik).  The chart's fp32 patterns are non-negative and
 //   order like unsigned integers, so c is found by a weighted radix select:
 //   every block adds its entries' probe weights into a global histogram of
-//   bits [30:19] (barrier B1), every block finds the bin where the weight
-//   counted from the top reaches K and lists its entries of that bin
-//   (barrier B2); every block then resolves bits [18:0] over the gathered
-//   candidates (or, with too many candidates, by two more grid-wide
-//   histogram passes).
+//   bits [30:19], writes its entries grouped by that digit into its own
+//   segment of the scratch and, per digit it holds, a descriptor (first
+//   slot, count) into a [digit][block] table (barrier B1).  Every block then
+//   finds the bin where the weight counted from the top reaches K, reads
+//   that bin's row of descriptors and, through them, the bin's entries from
+//   all segments, and resolves bits [18:0] over them in shared memory (with
+//   more candidates than fit, by two more grid-wide histogram passes).  One
+//   grid barrier in the common case.
 //
 //   Work split.  Block b streams output panel p = b mod P for the rows
 //   i = b / P + k nbp (nbp blocks share a panel; rows interleave so the
 //   heavy rows of a vector spread over the blocks).  Each (row, panel) is a
-//   work unit.  The units' list records are loaded while B1 fills, their
-//   stored chunks' first magnitudes while B2 fills.
+//   work unit.  The units' list records and their stored chunks' first
+//   magnitudes are loaded while B1 fills.
 //
 //   Dispatch (row a3).  Once c is known: for every unit the threshold
 //   tau_i(c), the smallest fp16 magnitude m with fl32(|v_i| m) >= c (|w| >=
@@ -48,7 +51,7 @@
 //   that sum |v_i| * max |w|, which bounds every partial sum, stays below 2^30
 //   units; each fp32 product is rounded once to the unit.  Each block adds
 //   its panel sums into out with float4 reductions (out was cleared by its
-//   column owners before B2); the last block to finish (a counter, no wait)
+//   column owners before B1); the last block to finish (a counter, no wait)
 //   publishes |S| and resets the scratch words.  The order of the fp32
 //   additions into out varies from call to call, so out is reproducible to
 //   rounding, c, |S| and the L_i bit for bit.
@@ -319,7 +322,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ 
 
   // ---- prologue: prepared-matrix data and shared memory only
   for (int e = tid; e < chs; e += kThreads) S.chart[e] = hd.probes[(size_t)r0 * kP + e];
-  for (int e = tid; e < V * kBins0; e += kThreads) S.hist[e] = 0u;
+  for (int e = tid; e < V * kBins0; e += kThreads) {
+    S.hist[e] = 0u;
+    reinterpret_cast<unsigned*>(S.cand)[e] = 0u;
+  }
   for (int e = tid; e < kBins1 + kBins2; e += kThreads) S.hist2[e] = 0u;
   for (int e = tid; e < V * kPW; e += kThreads) S.iacc[e] = 0;
   if (tid < 256) S.ctl[tid] = 0u;
@@ -386,45 +392,100 @@ __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ 
   __syncthreads();
 
   float c[V];
-  unsigned vsum_bits[V];
+  unsigned vsum_bits[V], b1[V], K1[V];  // b1, K1: crossing bin of the first digit, rank left inside it
 #pragma unroll
   for (int k = 0; k < V; ++k) {
     c[k] = 0.0f;
-    vsum_bits[k] = 0u;
+    vsum_bits[k] = b1[k] = K1[k] = 0u;
   }
   if (mode == kModeSelect) {
-    // ---- phase 1: charts and first-digit histograms
-    for (int e = tid; e < chs; e += kThreads) {
-      const unsigned w = (unsigned)hd.pw[e & (kP - 1)];
-      const unsigned pb = S.chart[e];  // probe bits, replaced by vector 0's chart
+    // ---- phase 1: charts, first-digit histograms, entries grouped by bin
+    unsigned* hcnt = reinterpret_cast<unsigned*>(S.cand);  // [V][kBins0] entries per bin, then (start << 16) | count
+    unsigned short* rank = reinterpret_cast<unsigned short*>(S.cidx);  // [V][chs] entry's place inside its bin
+    // entry e is probe e mod kP of its row, and kThreads is a multiple of kP:
+    // every entry this thread visits has the same probe weight
+    const unsigned w = (unsigned)hd.pw[tid & (kP - 1)];
+    if (w)
+      for (int e = tid; e < chs; e += kThreads) {
+        const unsigned pb = S.chart[e];  // probe bits, replaced by vector 0's chart
 #pragma unroll
-      for (int k = V - 1; k >= 0; --k) {
-        const unsigned xb = __float_as_uint(__fmul_rn(S.absv[k * rp + (e >> 4)], h2f(pb)));
-        S.chart[k * rp * kP + e] = xb;
-        if (w) atomicAdd(&S.hist[k * kBins0 + (xb >> 19)], w);
+        for (int k = V - 1; k >= 0; --k) {
+          const unsigned xb = __float_as_uint(__fmul_rn(S.absv[k * rp + (e >> 4)], h2f(pb)));
+          S.chart[k * rp * kP + e] = xb;
+          atomicAdd(&S.hist[k * kBins0 + (xb >> 19)], w);
+          rank[k * chs + e] = (unsigned short)atomicAdd(&hcnt[k * kBins0 + (xb >> 19)], 1u);
+        }
+      }
+    else
+      for (int e = tid; e < chs; e += kThreads) {
+        const unsigned pb = S.chart[e];
+#pragma unroll
+        for (int k = V - 1; k >= 0; --k)
+          S.chart[k * rp * kP + e] = __float_as_uint(__fmul_rn(S.absv[k * rp + (e >> 4)], h2f(pb)));
+      }
+    __syncthreads();
+    // each bin's first slot in the block's segment (bins in ascending order)
+#pragma unroll
+    for (int k = 0; k < V; ++k) {
+      constexpr int kQ0 = kBins0 / kThreads;
+      unsigned cq[kQ0], sum = 0, total = 0;
+#pragma unroll
+      for (int q = 0; q < kQ0; ++q) {
+        cq[q] = hcnt[k * kBins0 + tid * kQ0 + q];
+        sum += cq[q];
+      }
+      unsigned at = block_prefix_excl(sum, wsum, &total);
+#pragma unroll
+      for (int q = 0; q < kQ0; ++q) {
+        hcnt[k * kBins0 + tid * kQ0 + q] = (at << 16) | cq[q];
+        at += cq[q];
       }
     }
     __syncthreads();
+    // the weighted entries into the block's segment, grouped by bin (the
+    // order inside a bin is the order of the counting atomics; it does not
+    // matter), then the global histogram and this block's bin descriptors
+    if (w)
+      for (int e = tid; e < chs; e += kThreads)
+#pragma unroll
+        for (int k = 0; k < V; ++k) {
+          const unsigned xb = S.chart[k * rp * kP + e];
+          const unsigned slot = (hcnt[k * kBins0 + (xb >> 19)] >> 16) + rank[k * chs + e];
+          wsv[k].seg[(size_t)b * rp * kP + slot] = make_uint2(xb, w);
+        }
 #pragma unroll
     for (int k = 0; k < V; ++k)
       for (int e = tid; e < kBins0; e += kThreads) {
         const unsigned h = S.hist[k * kBins0 + e];
-        if (h) atomicAdd(&wsv[k].ghist0[e], h);
+        if (h) {
+          atomicAdd(&wsv[k].ghist0[e], h);
+          wsv[k].desc[(size_t)e * nb + b] = hcnt[k * kBins0 + e];
+        }
       }
     EFFORT_MARK(2);
     __syncthreads();
     if (tid == 0) grid_arrive_thread(ws.bar);
     ++nbar;
-    // while B1 fills: the first round's list records
-    for (int u = tid; u < nu0; u += kThreads) S.ulst[u] = hd.lst[(size_t)(j0 + u * nbp) * P + p];
+    // while B1 fills (thread 0 waits): the first round's list records and the
+    // first 16 stored chunks' first magnitudes of each
+    if (warp > 0) {
+      for (int u = tid - 32; u < nu0; u += kThreads - 32) S.ulst[u] = hd.lst[(size_t)(j0 + u * nbp) * P + p];
+      // warps 1.. only (named barrier 1): 16 consecutive threads read one unit's heads
+      asm volatile("bar.sync 1, %0;" ::"r"(kThreads - 32) : "memory");
+      for (int e = tid - 32; e < nu0 * 16; e += kThreads - 32) {
+        const uint4 Lr = S.ulst[e >> 4];
+        const unsigned k = (unsigned)(e & 15);
+        S.uhead[e] = (k < Lr.y && EFFORT_IN_RANGE(Lr.x + k < hd.total_chunks, status)) ? hd.head[Lr.x + k]
+                                                                                        : (unsigned short)0;
+      }
+    }
     if (tid == 0)
       S.ctl[kCtlFlag] = grid_wait_thread(ws.bar, bar_base + (unsigned long long)nbar * bnb, status) ? 1u : 0u;
     __syncthreads();
     if (!S.ctl[kCtlFlag]) return;
     EFFORT_MARK(3);
 
-    // ---- phase 2: crossing bins, candidates
-    unsigned b1[V], K1[V];
+    // ---- phase 2: crossing bins
 #pragma unroll
     for (int k = 0; k < V; ++k) {
       constexpr int kQ0 = kBins0 / kThreads;
@@ -435,47 +496,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ 
       block_crossing<kQ0>(h0, (unsigned)Kv[k], wsum, S.ctl + kCtlCross);
       b1[k] = S.ctl[kCtlCross];
       K1[k] = S.ctl[kCtlCross + 1];
-      const unsigned* chart = S.chart + k * rp * kP;
-      for (int e0 = 0; e0 < chs; e0 += kThreads) {
-        const int e = e0 + tid;
-        bool in = false;
-        unsigned xb = 0, w = 0;
-        if (e < chs) {
-          xb = chart[e];
-          w = (unsigned)hd.pw[e & (kP - 1)];
-          in = w != 0 && (xb >> 19) == b1[k];
-        }
-        const unsigned bal = __ballot_sync(0xFFFFFFFFu, in);
-        if (bal) {
-          unsigned basei = 0;
-          if (lane == 0) basei = atomicAdd(wsv[k].hdr + kHdrCand, (unsigned)__popc(bal));
-          basei = __shfl_sync(0xFFFFFFFFu, basei, 0);
-          const unsigned pos = basei + __popc(bal & ((1u << lane) - 1u));
-          if (in && pos < (unsigned)kCandCap) wsv[k].cand[pos] = make_uint2(xb, w);
-        }
-      }
     }
-    EFFORT_MARK(4);
-    __syncthreads();
-    if (tid == 0) grid_arrive_thread(ws.bar);
-    ++nbar;
-    // while B2 fills: the stored chunks' first magnitudes of the first round
-    for (int e = tid; e < nu0 * 16; e += kThreads) {
-      const uint4 Lr = S.ulst[e >> 4];
-      const unsigned k = (unsigned)(e & 15);
-      S.uhead[e] = (k < Lr.y && EFFORT_IN_RANGE(Lr.x + k < hd.total_chunks, status)) ? hd.head[Lr.x + k]
-                                                                                        : (unsigned short)0;
-    }
-    if (tid == 0) S.ctl[kCtlFlag] = grid_wait_thread(ws.bar, bar_base + (unsigned long long)nbar * bnb, status) ? 1u : 0u;
-    __syncthreads();
-    if (!S.ctl[kCtlFlag]) return;
-    EFFORT_MARK(5);
+    // every block's descriptor of the crossing bin (thread t: block t's)
+    unsigned dsc[V];
+#pragma unroll
+    for (int k = 0; k < V; ++k) dsc[k] = ((unsigned)tid < nb) ? __ldcg(&wsv[k].desc[(size_t)b1[k] * nb + tid]) : 0u;
+    // this block's descriptors of the other bins are read by nobody: clear
+    // them for the next call (the crossing bin's row is cleared by the last
+    // block)
 #pragma unroll
     for (int k = 0; k < V; ++k)
-      // the first-digit histogram is read by nobody any more: clear this block's share
-      for (int e = b * (kBins0 / 4) / (int)nb * 4 + tid, e1 = (b + 1) * (kBins0 / 4) / (int)nb * 4; e < e1;
-           e += kThreads)
-        wsv[k].ghist0[e] = 0u;
+      for (int e = tid; e < kBins0; e += kThreads)
+        if (S.hist[k * kBins0 + e] && (unsigned)e != b1[k]) wsv[k].desc[(size_t)e * nb + b] = 0u;
+    EFFORT_MARK(4);
 
     // ---- phase 3: bits [18:0] of each c
 #pragma unroll
@@ -491,18 +524,37 @@ __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ 
         for (int e = tid; e < kBins1 + kBins2; e += kThreads) S.hist2[e] = 0u;
         __syncthreads();
       }
-      // the first 2 kThreads candidates are loaded with the count (the common case)
-      const uint2 cA = __ldcg(&w_.cand[tid]), cB = __ldcg(&w_.cand[tid + kThreads]);
-      const unsigned M = __ldcg(w_.hdr + kHdrCand);
+      // the crossing bin's entries, from the blocks' segments through their
+      // descriptors
+      unsigned* gpos = reinterpret_cast<unsigned*>(S.cunit);  // [nb + 1] first candidate of each block
+      unsigned* gsrc = gpos + (nb + 1);                        // [nb] its first slot in the block's segment
+      unsigned M = 0;
+      const unsigned at = block_prefix_excl(dsc[k] & 0xFFFFu, wsum, &M);
+      if ((unsigned)tid < nb) {
+        gpos[tid] = at;
+        gsrc[tid] = dsc[k] >> 16;
+      }
+      if (tid == 0) gpos[nb] = M;
+      __syncthreads();
       if (M <= (unsigned)kCandCap) {
-        if ((unsigned)tid < M) S.cand[tid] = cA;
-        if ((unsigned)(tid + kThreads) < M) S.cand[tid + kThreads] = cB;
-        for (unsigned e0 = 2 * kThreads; e0 < M; e0 += 4 * kThreads) {
+        for (unsigned e0 = 0; e0 < M; e0 += 4 * kThreads) {
           uint2 t4[4];
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             const unsigned e = e0 + q * kThreads + tid;
-            t4[q] = (e < M) ? __ldcg(&w_.cand[e]) : make_uint2(0u, 0u);
+            t4[q] = make_uint2(0u, 0u);
+            if (e < M) {
+              // the block holding candidate e: the last one whose first candidate is <= e
+              unsigned lo = 0, hi = nb - 1;
+              while (lo < hi) {
+                const unsigned mid = (lo + hi + 1) >> 1;
+                if (gpos[mid] <= e) lo = mid;
+                else hi = mid - 1;
+              }
+              const unsigned slot = gsrc[lo] + (e - gpos[lo]);
+              if (EFFORT_IN_RANGE(slot < (unsigned)(rp * kP), status))
+                t4[q] = __ldcg(&w_.seg[(size_t)lo * rp * kP + slot]);
+            }
           }
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
@@ -510,6 +562,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ 
             if (e < M) S.cand[e] = t4[q];
           }
         }
+        EFFORT_MARK(5);
         __syncthreads();
         for (unsigned e = tid; e < M; e += kThreads) atomicAdd(&h1[(S.cand[e].x >> 9) & (kBins1 - 1)], S.cand[e].y);
         __syncthreads();
@@ -536,7 +589,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ 
       } else {
         // too many candidates for one block: two more grid-wide histogram passes
         for (int e = tid; e < chs; e += kThreads) {
-          const unsigned xb = chart[e], w = (unsigned)hd.pw[e & (kP - 1)];
+          const unsigned xb = chart[e];
           if (w && (xb >> 19) == b1[k]) atomicAdd(&h1[(xb >> 9) & (kBins1 - 1)], w);
         }
         __syncthreads();
@@ -553,7 +606,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ 
         b2 = S.ctl[kCtlCross];
         const unsigned K2 = S.ctl[kCtlCross + 1];
         for (int e = tid; e < chs; e += kThreads) {
-          const unsigned xb = chart[e], w = (unsigned)hd.pw[e & (kP - 1)];
+          const unsigned xb = chart[e];
           if (w && (xb >> 19) == b1[k] && ((xb >> 9) & (kBins1 - 1)) == b2) atomicAdd(&h2[xb & (kBins2 - 1)], w);
         }
         __syncthreads();
@@ -956,7 +1009,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ 
         const unsigned long long cnt = count_all[k] ? hd.kept_total : __ldcg(wsv[k].count);
         if (cntp[k]) *cntp[k] = cnt;
         *wsv[k].count = 0ull;
-        wsv[k].hdr[kHdrCand] = 0u;
         wsv[k].hdr[kHdrVsum] = 0u;
       }
       ws.hdr[kHdrDone] = 0u;
@@ -967,11 +1019,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ 
       run[0] = 0ull;
       run[1] = 0ull;
     }
-    // the last digit's histograms of the many-candidates path are read by nobody any more
+    // the first-digit histograms, the crossing bins' descriptors and the last
+    // digit's histograms of the many-candidates path are read by nobody any more
     if (mode == kModeSelect)
 #pragma unroll
-      for (int k = 0; k < V; ++k)
+      for (int k = 0; k < V; ++k) {
+        for (int e = tid; e < kBins0; e += kThreads) wsv[k].ghist0[e] = 0u;
+        for (int e = tid; e < (int)nb; e += kThreads) wsv[k].desc[(size_t)b1[k] * nb + e] = 0u;
         for (int e = tid; e < kBins2; e += kThreads) wsv[k].ghist2[e] = 0u;
+      }
     // every block has added its sums: the finished out to host memory
     if (jb.out_mirror)
       for (int j = tid; j < O; j += kThreads) jb.out_mirror[j] = __ldcg(jb.out + j);

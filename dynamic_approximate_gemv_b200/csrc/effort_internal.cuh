@@ -61,6 +61,13 @@ enum : unsigned { kStatusNonfiniteV = 1u, kStatusNonfiniteW = 2u, kStatusInterna
 // radix-select digits of the non-negative fp32 chart: bits [30:19], [18:9], [8:0]
 constexpr int kBins0 = 4096, kBins1 = 1024, kBins2 = 512;
 constexpr int kCandCap = 4096;     // crossing-bin candidates resolved in one block's shared memory
+constexpr int kMaxGrid = 512;      // blocks of a matvec grid (one per SM) the crossing-bin gather handles
+// chart entries of one block: 16-bit offsets in the bin descriptors, and the
+// ranks of two charts' entries share the chunk-index area
+constexpr int kMaxSegEntries = kChunkCap;
+static_assert(kMaxSegEntries <= 65535 && 2 * kMaxSegEntries * 2 <= kChunkCap * 4, "segment entry bound");
+static_assert(2 * kBins0 * 4 <= kCandCap * 8, "two charts' bin counts share the candidate area");
+static_assert(2 * (kMaxGrid + 1) * 4 <= kChunkCap * 2, "the gather offsets share the chunk-unit area");
 
 // Device-resident description of a prepared matrix (passed by value).
 struct HandleDesc {
@@ -77,8 +84,8 @@ struct HandleDesc {
   int pw[kP];              // probe weights (entries each probe stands for)
 };
 
-// Per-call scratch in device memory.  The header words and the first-digit
-// histogram must be zero before a call (the library clears them at
+// Per-call scratch in device memory.  The header words, the histograms and
+// the bin descriptors must be zero before a call (the library clears them at
 // allocation and every call leaves them zero, except after a timeout).
 struct WsPtrs {
   unsigned* hdr;              // see kHdr* below
@@ -87,14 +94,14 @@ struct WsPtrs {
   unsigned* ghist0;           // [kBins0]
   unsigned* ghist1;           // [kBins1]
   unsigned* ghist2;           // [kBins2]
-  uint2* cand;                // [kCandCap] {chart bits, weight}
+  unsigned* desc;             // [kBins0][grid]: block b's entries of first-digit bin h, (start << 16) | count
+  uint2* seg;                 // [grid][rows_per_block * kP]: block b's chart entries {bits, weight}, grouped by bin
 };
-// header words: status, candidate count, then 64-bit byte counters: the dense
-// and sparse bytes the running call plans to read (words 8..11) and those of
-// the last finished call (words 12..15)
+// header words: status, (unused), finished blocks, then 64-bit byte counters:
+// the dense and sparse bytes the running call plans to read (words 8..11) and
+// those of the last finished call (words 12..15)
 // (word 3: the running sum of |v| over the blocks, fp32 bits)
-enum : int { kHdrStatus = 0, kHdrCand = 1, kHdrDone = 2, kHdrVsum = 3, kHdrBytesRun = 8, kHdrBytesLast = 12,
-             kHdrWords = 64 };
+enum : int { kHdrStatus = 0, kHdrDone = 2, kHdrVsum = 3, kHdrBytesRun = 8, kHdrBytesLast = 12, kHdrWords = 64 };
 
 struct Job {
   HandleDesc hd;
@@ -146,14 +153,16 @@ __host__ __device__ inline SmemLayout smem_layout(int I, int nb, int V = 1) {
   L.absv = take((size_t)V * rp * 4);                  // |v| of the cutoff rows
   L.hist = take((size_t)V * kBins0 * 4);              // first-digit histograms
   L.hist2 = take((size_t)(kBins1 + kBins2) * 4);      // second- and third-digit histograms
-  L.cand = take((size_t)kCandCap * 8);                // gathered candidates
+  L.cand = take((size_t)kCandCap * 8);                // per-bin entry counts of the charts, then the
+                                                      // gathered crossing-bin candidates
   L.ulst = take((size_t)kUnitCap * 16);               // list records of the round's (row, panel) units
   L.uhead = take((size_t)kUnitCap * 32);              // their first 16 stored chunks' first magnitudes
   L.uv = take((size_t)V * kUnitCap * 4);              // v of the unit's row
   L.utau = take((size_t)V * kUnitCap * 4);            // threshold of the unit's row
   L.dlist = take((size_t)kUnitCap * 2);               // units read dense
   L.cidx = take((size_t)kChunkCap * 4);               // sparse chunks to read (chunk index)
-  L.cunit = take((size_t)kChunkCap * 2);              // and the unit of each
+  L.cunit = take((size_t)kChunkCap * 2);              // and the unit of each (before the dispatch: the
+                                                      // crossing-bin gather's per-block offsets)
   L.ctl = take(256 * 4);                              // control words
   L.total = o;
   return L;

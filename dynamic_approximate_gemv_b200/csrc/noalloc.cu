@@ -25,7 +25,7 @@
 
 namespace effort {
 size_t handle_scratch_bytes(effort_handle_t h);
-size_t handle_scratch_zero_bytes();
+size_t handle_scratch_zero_bytes(effort_handle_t h);
 WsPtrs handle_carve(effort_handle_t h, char* base);
 int handle_device(effort_handle_t h);
 effort_status_t handle_fill_job(effort_handle_t h, const WsPtrs& ws, const void* v, effort_dtype_t v_dtype,
@@ -127,9 +127,10 @@ extern "C" effort_status_t effort_gemv_static(effort_handle_t h, const void* v, 
   st = handle_fill_job(h, ws, v, v_dtype, effort, out, cutoff_out, count_out, &job);
   if (st != EFFORT_OK) return st;
   cudaStream_t s = (cudaStream_t)stream;
-  // header, barrier counter and histograms start at zero; everything else is
-  // written before it is read within the call
-  cudaError_t e = cudaMemsetAsync(base, 0, handle_scratch_zero_bytes(), s);
+  // header, barrier counter, histograms and bin descriptors start at zero
+  // (whatever an earlier call on this device left, a timed-out one
+  // included); everything else is written before it is read within the call
+  cudaError_t e = cudaMemsetAsync(base, 0, handle_scratch_zero_bytes(h), s);
   if (e == cudaSuccess) e = handle_launch(h, job, s);
   if (e == cudaSuccess && status_out)
     e = cudaMemcpyAsync(status_out, ws.hdr + kHdrStatus, 4, cudaMemcpyDeviceToDevice, s);

@@ -54,7 +54,7 @@ typedef enum { EFFORT_F32 = 0, EFFORT_F16 = 1 } effort_dtype_t;
 /* Size limits of this build. */
 #define EFFORT_MAX_OUT_DIM 32768      /* a row is sorted inside one thread block */
 #define EFFORT_MAX_IN_DIM 40960       /* a block's share of the chart lives in its shared memory */
-#define EFFORT_STATIC_SCRATCH_BYTES (2u << 20) /* per-device scratch of effort_gemv_static */
+#define EFFORT_STATIC_SCRATCH_BYTES (8u << 20) /* per-device scratch of effort_gemv_static */
 
 /*
  * effort_prepare -- the offline pass: `precompute(W)` of the pages.
@@ -162,7 +162,7 @@ effort_status_t effort_grid_blocks(effort_handle_t h, int32_t* blocks);
 
 /*
  * effort_gemv_static -- effort_gemv_ex (without rowlen_out) whose per-call
- *   scratch is a fixed array of EFFORT_STATIC_SCRATCH_BYTES (2 MiB) per device,
+ *   scratch is a fixed array of EFFORT_STATIC_SCRATCH_BYTES (8 MiB) per device,
  *   compiled into the library, instead of the handle's workspace.  The pages
  *   have no counterpart: this is a library service, not part of the method.
  *   It is for callers that must not allocate device memory on the call path,
@@ -184,9 +184,10 @@ effort_status_t effort_grid_blocks(effort_handle_t h, int32_t* blocks);
  *     GPU (unordered streams, concurrent host threads) race and give wrong
  *     results; order them on one stream.
  *   Returns EFFORT_ERR_UNSUPPORTED when the handle's geometry needs more than
- *     EFFORT_STATIC_SCRATCH_BYTES of scratch (every geometry this build
- *     supports needs the same 55 KiB: histograms, candidates and a header),
- *     and when the device ordinal is 64 or above.
+ *     EFFORT_STATIC_SCRATCH_BYTES of scratch (a geometry needs about 2.4 MiB
+ *     of histograms and bin descriptors on a 148-SM device plus 128 bytes per
+ *     input row for the chart entries: 3.0 MiB at in_dim 4096, 7.7 MiB at
+ *     EFFORT_MAX_IN_DIM), and when the device ordinal is 64 or above.
  *   The array's address is looked up again whenever the device's primary
  *     context has changed (after cudaDeviceReset), never kept across it.
  */
