@@ -88,7 +88,7 @@ __device__ __forceinline__ bool passes(float a, unsigned m, float x) { return __
 __device__ __forceinline__ unsigned tau_of(float a, float x) {
   if (!(x > 0.0f)) return 0u;
   if (!passes(a, 0x7BFFu, x)) return 0x7C00u;
-  unsigned m = __half_as_ushort(__float2half_rn(x / a)) & 0x7FFFu;
+  unsigned m = __half_as_ushort(__float2half_rn(__fdividef(x, a))) & 0x7FFFu;  // a guess: the tests below decide
   if (m > 0x7BFFu) m = 0x7BFFu;
 #pragma unroll 1
   for (int k = 0; k < 4 && m > 0 && passes(a, m - 1, x); ++k) --m;
@@ -218,7 +218,11 @@ __device__ __forceinline__ void block_crossing(const unsigned (&h)[Q], unsigned 
 enum : int {
   kCtlFlag = 0, kCtlCross = 2, kCtlWsum = 8,  // kCtlWsum: kWarps words
   kCtlC = 40, kCtlSc = 41, kCtlInvSc = 42, kCtlLast = 43, kCtlExtraDense = 44, kCtlChunks = 45,
+  kCtlCounts = 48,  // 2 kWarps 64-bit words: per-warp used counts
 };
+// the call's 64-bit count word: |S| of vector 0 in bits [39:0], finished
+// blocks above
+constexpr int kArrivalShift = 40;
 
 struct KSmem {
   int* iacc;
@@ -238,11 +242,17 @@ struct KSmem {
 };
 
 // Stored chunks of a list whose first magnitude reaches tau: the first 16
-// heads come from shared memory, any further ones from the prepared matrix.
+// heads come from shared memory (two 16-byte reads, compared two at a time;
+// the slots past the list's stored chunks hold 0 and are not counted), any
+// further ones from the prepared matrix.
 __device__ __forceinline__ unsigned chunks_reaching(const HandleDesc& hd, const uint4& Lr, const unsigned short* uh,
                                                     unsigned tau, unsigned* status) {
-  unsigned m = 0;
-  for (unsigned k = 0; k < Lr.y && k < 16u; ++k) m += (uh[k] >= tau) ? 1u : 0u;
+  const uint4 ha = reinterpret_cast<const uint4*>(uh)[0], hb = reinterpret_cast<const uint4*>(uh)[1];
+  const unsigned t2 = tau | (tau << 16);
+  const unsigned bits = __popc(__vcmpgeu2(ha.x, t2)) + __popc(__vcmpgeu2(ha.y, t2)) + __popc(__vcmpgeu2(ha.z, t2)) +
+                        __popc(__vcmpgeu2(ha.w, t2)) + __popc(__vcmpgeu2(hb.x, t2)) + __popc(__vcmpgeu2(hb.y, t2)) +
+                        __popc(__vcmpgeu2(hb.z, t2)) + __popc(__vcmpgeu2(hb.w, t2));
+  unsigned m = min(bits >> 4, min(Lr.y, 16u));
   for (unsigned k = 16; k < Lr.y; ++k)
     if (EFFORT_IN_RANGE(Lr.x + k < hd.total_chunks, status)) m += (hd.head[Lr.x + k] >= tau) ? 1u : 0u;
   (void)status;
@@ -343,6 +353,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ 
   // blocks already at this call's first barrier (fewer than nb)
   const unsigned long long bar_base = (__ldcg(ws.bar) / nb) * nb;
   int nbar = 0;  // grid barriers of this call so far
+  // the last-call byte words start over (the blocks add to them at the end,
+  // after at least one grid barrier)
+  if (b == 0 && tid == 0 && !jb.accumulate_bytes) {
+    unsigned long long* last = reinterpret_cast<unsigned long long*>(ws.hdr + kHdrBytesLast);
+    last[0] = 0ull;
+    last[1] = 0ull;
+  }
 
   const int oc0 = (int)((long long)O * b / nb), oc1 = (int)((long long)O * (b + 1) / nb);  // this block's columns
 
@@ -981,44 +998,55 @@ __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ 
   }
   EFFORT_MARK(11);
 
-  // ---- used counts and planned bytes; the last block to finish publishes them
+  // ---- used counts and planned bytes.  The block's count of vector 0 and
+  // its arrival go into one 64-bit counter (arrivals in bits [63:40]), so
+  // the block that arrives last gets the total with its own atomic; the
+  // planned bytes go straight into the last-call words (cleared before the
+  // first barrier unless the call accumulates them).
+  unsigned long long* wcnt = reinterpret_cast<unsigned long long*>(S.ctl + kCtlCounts);  // [V][kWarps]
 #pragma unroll
   for (int k = 0; k < V; ++k) {
     unsigned long long x = my_count[k];
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xFFFFFFFFu, x, o);
-    if (lane == 0 && x && !count_all[k]) atomicAdd(wsv[k].count, x);
+    if (lane == 0) wcnt[k * kWarps + warp] = count_all[k] ? 0ull : x;
   }
   if (tid == 0) {
-    unsigned long long* run = reinterpret_cast<unsigned long long*>(ws.hdr + kHdrBytesRun);
-    if (planned_dense) atomicAdd(run, planned_dense);
-    if (planned_sparse) atomicAdd(run + 1, planned_sparse);
+    unsigned long long* last = reinterpret_cast<unsigned long long*>(ws.hdr + kHdrBytesLast);
+    if (planned_dense) atomicAdd(last, planned_dense);
+    if (planned_sparse) atomicAdd(last + 1, planned_sparse);
   }
   __syncthreads();
   if (tid == 0) {
+    unsigned long long mine[V];
+#pragma unroll
+    for (int k = 0; k < V; ++k) {
+      mine[k] = 0ull;
+      for (int q = 0; q < kWarps; ++q) mine[k] += wcnt[k * kWarps + q];
+    }
+#pragma unroll
+    for (int k = 1; k < V; ++k)
+      if (mine[k]) atomicAdd(wsv[k].count, mine[k]);
     __threadfence();
-    const unsigned arrived = atomicAdd(ws.hdr + kHdrDone, 1u);
-    S.ctl[kCtlLast] = (arrived == nb - 1u) ? 1u : 0u;
-  }
-  __syncthreads();
-  if (S.ctl[kCtlLast]) {
-    __threadfence();
-    if (tid == 0) {
+    const unsigned long long add = (1ull << kArrivalShift) | mine[0];
+    const unsigned long long before = atomicAdd(ws.count, add);
+    const bool is_last = (before >> kArrivalShift) == (unsigned long long)(nb - 1u);
+    S.ctl[kCtlLast] = is_last ? 1u : 0u;
+    if (is_last) {
+      __threadfence();
+      const unsigned long long total0 = (before + add) & ((1ull << kArrivalShift) - 1ull);
 #pragma unroll
       for (int k = 0; k < V; ++k) {
-        const unsigned long long cnt = count_all[k] ? hd.kept_total : __ldcg(wsv[k].count);
+        const unsigned long long cnt = count_all[k] ? hd.kept_total : (k == 0 ? total0 : __ldcg(wsv[k].count));
         if (cntp[k]) *cntp[k] = cnt;
         *wsv[k].count = 0ull;
         wsv[k].hdr[kHdrVsum] = 0u;
       }
-      ws.hdr[kHdrDone] = 0u;
-      unsigned long long* run = reinterpret_cast<unsigned long long*>(ws.hdr + kHdrBytesRun);
-      unsigned long long* last = reinterpret_cast<unsigned long long*>(ws.hdr + kHdrBytesLast);
-      last[0] = (jb.accumulate_bytes ? __ldcg(last) : 0ull) + __ldcg(run);
-      last[1] = (jb.accumulate_bytes ? __ldcg(last + 1) : 0ull) + __ldcg(run + 1);
-      run[0] = 0ull;
-      run[1] = 0ull;
     }
+  }
+  __syncthreads();
+  if (S.ctl[kCtlLast]) {
+    __threadfence();
     // the first-digit histograms, the crossing bins' descriptors and the last
     // digit's histograms of the many-candidates path are read by nobody any more
     if (mode == kModeSelect)

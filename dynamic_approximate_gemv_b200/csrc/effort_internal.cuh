@@ -90,18 +90,17 @@ struct HandleDesc {
 struct WsPtrs {
   unsigned* hdr;              // see kHdr* below
   unsigned long long* bar;    // grid-barrier counter (monotonic)
-  unsigned long long* count;  // running |S|
+  unsigned long long* count;  // running |S| (vector 0's: bits [39:0], the finished blocks above)
   unsigned* ghist0;           // [kBins0]
   unsigned* ghist1;           // [kBins1]
   unsigned* ghist2;           // [kBins2]
   unsigned* desc;             // [kBins0][grid]: block b's entries of first-digit bin h, (start << 16) | count
   uint2* seg;                 // [grid][rows_per_block * kP]: block b's chart entries {bits, weight}, grouped by bin
 };
-// header words: status, (unused), finished blocks, then 64-bit byte counters:
-// the dense and sparse bytes the running call plans to read (words 8..11) and
-// those of the last finished call (words 12..15)
-// (word 3: the running sum of |v| over the blocks, fp32 bits)
-enum : int { kHdrStatus = 0, kHdrDone = 2, kHdrVsum = 3, kHdrBytesRun = 8, kHdrBytesLast = 12, kHdrWords = 64 };
+// header words: status (word 0), the running sum of |v| over the blocks
+// (word 3, fp32 bits), and the 64-bit dense and sparse bytes the last call
+// planned to read (words 12..15, added up by the blocks as they finish)
+enum : int { kHdrStatus = 0, kHdrVsum = 3, kHdrBytesLast = 12, kHdrWords = 64 };
 
 struct Job {
   HandleDesc hd;
