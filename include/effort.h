@@ -145,8 +145,10 @@ effort_status_t effort_gemv_host(effort_handle_t h, const void* v_host, effort_d
  *   timing: marks is a device uint64 array [blocks][16] (blocks from
  *   effort_grid_blocks); entry k of block b is written by that block when it
  *   reaches point k: 0 start, 1 after waiting for the preceding grid, 2 chart
- *   histogram pushed, 3 after the first grid barrier, 4 candidates listed,
- *   5 after the second grid barrier, 6 cutoff resolved, 7 work lists built,
+ *   histogram, entries and bin descriptors written, 3 after the first grid
+ *   barrier, 4 crossing bin found, 5 the crossing bin's entries gathered
+ *   (not reached with more than 4096 of them), 6 cutoff resolved, 7 work
+ *   lists built,
  *   8 dense units streamed, 9 sparse chunks streamed, 10 registers added into
  *   the panel accumulator, 11 the block's sums added into out, 13 the block is
  *   done (12, 14 and 15 are not used); 8 and 9 are written by lane 0 of every
