@@ -35,3 +35,18 @@ def gate(n_experts, in_dim, seed, scale=1.0 / 64):
     """Router matrix [n_experts x in_dim] float32, N(0, 1) * scale."""
     rng = np.random.default_rng(seed)
     return (rng.standard_normal((n_experts, in_dim)) * scale).astype(np.float32)
+
+
+def q8_weights(in_dim, out_dim, seed, sigma=SIGMA_W):
+    """Q8 weights of the same draw as `weights`: (q int8 [in_dim x out_dim],
+    s float16 [in_dim]) with s_i = fp16(max_j |w_ij| / 127) and q_ij =
+    round(w_ij / s_i) clipped to [-127, 127] (per-row symmetric absmax
+    quantisation of a N(0, sigma^2) float32 draw).  A row that is all zero
+    gets s_i = 1."""
+    rng = np.random.default_rng(seed)
+    w = rng.standard_normal((in_dim, out_dim), dtype=np.float32) * np.float32(sigma)
+    amax = np.abs(w).max(axis=1)
+    s = (amax / np.float32(127.0)).astype(np.float16)
+    s[s == 0] = np.float16(1.0)
+    q = np.clip(np.rint(w / s.astype(np.float32)[:, None]), -127, 127).astype(np.int8)
+    return q, s
