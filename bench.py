@@ -255,18 +255,27 @@ def read_bytes(in_dim, out_dim, dense, sparse, v_bytes=4):
 
 
 # ----------------------------------------------------------------- other shapes
-def measure_shape(E, dev, in_dim, out_dim, efforts, dist, n_mats=10, n_vecs=8, seed0=5000, keep=1.0):
+def measure_shape(E, dev, in_dim, out_dim, efforts, dist, n_mats=10, n_vecs=8, seed0=5000, keep=1.0, q8=False):
     """us per matvec and algorithmic GB/s on another workload shape: n_mats
     prepared matrices N(0, 0.02^2) fp16 and n_vecs vectors rotated through CUDA
-    graphs of 40 steps (inputs larger than L2), as for the headline workload."""
+    graphs of 40 steps (inputs larger than L2), as for the headline workload.
+    q8: the same draws quantised per row to int8 with a binary16 scale
+    (s_i = fp16(max |w_i| / 127), q = round(w / s_i) clipped to +-127)."""
     import torch
     from dynamic_approximate_gemv_b200 import inputs
     g = torch.Generator(device=dev)
     mats = []
     for m in range(n_mats):
         g.manual_seed(seed0 + m)
-        W = (torch.randn(in_dim, out_dim, device=dev, generator=g) * 0.02).to(torch.float16)
-        mats.append(E.PreparedMatrix(W, keep))
+        W = torch.randn(in_dim, out_dim, device=dev, generator=g) * 0.02
+        if q8:
+            sc = (W.abs().amax(dim=1) / 127.0).to(torch.float16)
+            sc[sc == 0] = 1.0
+            q = torch.clamp(torch.round(W / sc.float()[:, None]), -127, 127).to(torch.int8)
+            mats.append(E.PreparedMatrix.from_q8(q, sc, keep))
+            del q, sc
+        else:
+            mats.append(E.PreparedMatrix(W.to(torch.float16), keep))
         del W
     vecs = [torch.from_numpy(inputs.vector(in_dim, seed0 + 100 + k, dist)).to(dev) for k in range(n_vecs)]
     outs = [torch.empty(out_dim, device=dev) for _ in range(n_mats)]
@@ -305,9 +314,15 @@ def measure_shape(E, dev, in_dim, out_dim, efforts, dist, n_mats=10, n_vecs=8, s
         e1.record()
         torch.cuda.synchronize()
         us = e0.elapsed_time(e1) * 1000.0 / (reps * steps)
-        b = algorithmic_bytes(in_dim, out_dim, used)
-        rb = read_bytes(in_dim, out_dim, dense, sparse)
-        dense_b = 2.0 * in_dim * out_dim + 4.0 * in_dim + 4.0 * out_dim
+        if q8:
+            # 2 bytes per used product (int8 value and an 8-bit position), probes, row scales, v, out
+            b = algorithmic_bytes(in_dim, out_dim, used) - used + 2.0 * in_dim
+            rb = read_bytes(in_dim, out_dim, dense, sparse) + 2.0 * in_dim
+            dense_b = 1.0 * in_dim * out_dim + 2.0 * in_dim + 4.0 * in_dim + 4.0 * out_dim
+        else:
+            b = algorithmic_bytes(in_dim, out_dim, used)
+            rb = read_bytes(in_dim, out_dim, dense, sparse)
+            dense_b = 2.0 * in_dim * out_dim + 4.0 * in_dim + 4.0 * out_dim
         res[str(e)] = {"us": us, "gbs_algorithmic": b / (us * 1e-6) / 1e9, "mean_used": used,
                        "read_bytes": {"dense": dense, "sparse": sparse, "total": rb},
                        "gbs_read": rb / (us * 1e-6) / 1e9,
@@ -811,6 +826,12 @@ def main():
         shapes["FFN down 14336x4096, v t3/sqrt(3)"] = measure_shape(E, dev, 14336, 4096, (0.25, 0.15), "t3")
         shapes["FFN up 4096x14336, keep 0.75, v t3/sqrt(3)"] = measure_shape(E, dev, 4096, 14336, (0.25, 0.15),
                                                                              "t3", keep=0.75)
+        # Q8 weights (row f3) on the headline shape; the int8 dense roofline is half the fp16 one
+        try:
+            shapes["Q8 FFN up 4096x14336, v t3/sqrt(3)"] = measure_shape(E, dev, 4096, 14336, (1.0, 0.5, 0.25, 0.15),
+                                                                         "t3", q8=True)
+        except Exception as ex:  # reported, not fatal: the headline line stands on its own
+            shapes["Q8 FFN up 4096x14336, v t3/sqrt(3)"] = {"error": repr(ex)[:200]}
 
     # the decode chain (one token through 32 layers)
     chain = measure_chain(E, dev) if (not a.no_sweep and world == 1) else {}

@@ -43,7 +43,7 @@ class Layout(ctypes.Structure):
                 ("n_probes", ctypes.c_int32), ("dense_stride", ctypes.c_int32), ("total_chunks", ctypes.c_uint32),
                 ("vals", ctypes.c_void_p), ("gaps", ctypes.c_void_p), ("head", ctypes.c_void_p),
                 ("lists", ctypes.c_void_p), ("wdense", ctypes.c_void_p), ("probes", ctypes.c_void_p),
-                ("scratch_bytes", ctypes.c_size_t)]
+                ("scratch_bytes", ctypes.c_size_t), ("weight_kind", ctypes.c_int32), ("scales", ctypes.c_void_p)]
 
 
 def lib():
@@ -57,6 +57,7 @@ def lib():
         vp, i64, i32, f32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float
         sig = {
             "effort_prepare": [vp, i64, i64, f32, vp, ctypes.POINTER(vp)],
+            "effort_prepare_q8": [vp, vp, i64, i64, f32, vp, ctypes.POINTER(vp)],
             "effort_gemv": [vp, vp, f32, vp, vp],
             "effort_gemv_ex": [vp, vp, ctypes.c_int, f32, vp, vp, vp, vp, vp],
             "effort_gemv_host": [vp, vp, ctypes.c_int, f32, vp, vp],
@@ -136,6 +137,28 @@ class PreparedMatrix:
             _check(lib().effort_prepare(_ptr(W), self.in_dim, self.out_dim, ctypes.c_float(keep_fraction),
                                         _stream(W.device), ctypes.byref(h)), "effort_prepare")
         self._h = h
+
+    @classmethod
+    def from_q8(cls, q, scales, keep_fraction=1.0):
+        """A Q8 matrix: int8 q [in_dim x out_dim] and float16 row scales
+        [in_dim] (w = scales[i] * q[i, j], exact), prepared for effort_gemv."""
+        _need_cuda(q, "q")
+        _need_cuda(scales, "scales")
+        if q.dtype != torch.int8 or q.dim() != 2:
+            raise ValueError("q must be a 2-D int8 tensor")
+        if scales.dtype != torch.float16 or tuple(scales.shape) != (q.shape[0],):
+            raise ValueError("scales must be float16 [in_dim]")
+        self = cls.__new__(cls)
+        self.in_dim, self.out_dim = q.shape
+        self.device = q.device
+        self.keep_fraction = float(keep_fraction)
+        h = ctypes.c_void_p()
+        with torch.cuda.device(q.device):
+            _check(lib().effort_prepare_q8(_ptr(q), _ptr(scales), self.in_dim, self.out_dim,
+                                           ctypes.c_float(keep_fraction), _stream(q.device), ctypes.byref(h)),
+                   "effort_prepare_q8")
+        self._h = h
+        return self
 
     def gemv(self, v, effort, out=None, cutoff=None, count=None, rowlen=None):
         """out[j] = sum over used (i, j) of v[i] * W[i, j]; returns out (fp32)."""
@@ -243,14 +266,18 @@ class PreparedMatrix:
         def view(ptr, shape, typestr):
             return torch.as_tensor(_CudaView(ptr, shape, typestr), device=self.device)
 
-        return {
+        vt = "|i1" if L.weight_kind == 1 else "<i2"  # int8 values of a Q8 matrix
+        out = {
             "n_kept": L.n_kept, "n_panels": P, "panel_width": L.panel_width, "chunk_slots": cs,
             "store_num": L.store_num, "store_den": L.store_den, "total_chunks": nc,
-            "dense_stride": L.dense_stride, "scratch_bytes": L.scratch_bytes,
-            "vals": view(L.vals, (max(nc, 1) * cs,), "<i2"), "gaps": view(L.gaps, (max(nc, 1) * cs,), "|u1"),
+            "dense_stride": L.dense_stride, "scratch_bytes": L.scratch_bytes, "weight_kind": L.weight_kind,
+            "vals": view(L.vals, (max(nc, 1) * cs,), vt), "gaps": view(L.gaps, (max(nc, 1) * cs,), "|u1"),
             "head": view(L.head, (max(nc, 1),), "<i2"), "lists": view(L.lists, (I, P, 4), "<u4"),
-            "wdense": view(L.wdense, (I, L.dense_stride), "<i2"), "probes": view(L.probes, (I, L.n_probes), "<i2"),
+            "wdense": view(L.wdense, (I, L.dense_stride), vt), "probes": view(L.probes, (I, L.n_probes), "<i2"),
         }
+        if L.weight_kind == 1:
+            out["scales"] = view(L.scales, (I,), "<i2")
+        return out
 
     def close(self):
         if getattr(self, "_h", None):

@@ -14,9 +14,9 @@
 #include "effort_internal.cuh"
 
 namespace effort {
-cudaError_t launch_prep(const uint16_t* W, int I, int O, int n, int P, int dstride, const int* prank,
-                        uint16_t* wdense, uint16_t* probes, uint16_t* vals, uint8_t* gaps, uint16_t* head, uint4* lst,
-                        unsigned* chunk_count, unsigned cap_chunks, unsigned* status, cudaStream_t stream);
+cudaError_t launch_prep(const void* W, const uint16_t* scales, int wk, int I, int O, int n, int P, int dstride,
+                        const int* prank, void* wdense, uint16_t* probes, void* vals, uint8_t* gaps, uint16_t* head,
+                        uint4* lst, unsigned* chunk_count, unsigned cap_chunks, unsigned* status, cudaStream_t stream);
 unsigned long long prep_chunk_bound_per_row(int O, int n);
 size_t effort_smem_bytes(int I, int nb);
 cudaError_t effort_kernel_attributes(int I, size_t smem);
@@ -267,27 +267,33 @@ const char* effort_status_string(effort_status_t s) {
   return "unknown status";
 }
 
-effort_status_t effort_prepare(const void* W, int64_t in_dim, int64_t out_dim, float keep_fraction, void* stream,
-                               effort_handle_t* out_handle) {
+// Both weight kinds: W is binary16 [in x out] (wk = kWeightF16), or int8
+// [in x out] with one binary16 scale per row (kWeightQ8).  esz: bytes of one
+// weight value.
+static effort_status_t prepare_impl(const void* W, const uint16_t* scales, int wk, int64_t in_dim, int64_t out_dim,
+                                    float keep_fraction, void* stream, effort_handle_t* out_handle) {
   if (!out_handle) return EFFORT_ERR_ARG;
   *out_handle = nullptr;
   if (!W || in_dim < 1 || out_dim < 1) return EFFORT_ERR_ARG;
-  if (((uintptr_t)W & 1u) != 0) return EFFORT_ERR_ARG;
+  if (wk == kWeightF16 && ((uintptr_t)W & 1u) != 0) return EFFORT_ERR_ARG;
+  if (wk == kWeightQ8 && (!scales || ((uintptr_t)scales & 1u) != 0)) return EFFORT_ERR_ARG;
   if (!(keep_fraction > 0.0f && keep_fraction <= 1.0f)) return EFFORT_ERR_ARG;
   if (out_dim > EFFORT_MAX_OUT_DIM || in_dim > EFFORT_MAX_IN_DIM) return EFFORT_ERR_UNSUPPORTED;
   if ((unsigned long long)in_dim * (unsigned long long)out_dim >= (1ull << 32)) return EFFORT_ERR_UNSUPPORTED;
   const int n = (int)floor((double)keep_fraction * (double)out_dim + 0.5);
   if (n < 1) return EFFORT_ERR_ARG;
+  const size_t esz = (wk == kWeightQ8) ? 1 : 2;
 
   // storage sizes need no device: check them against the allocation cap first
   const int I = (int)in_dim, O = (int)out_dim;
   const int P = (O + kPW - 1) / kPW, dstride = (O + kStripe - 1) / kStripe * kStripe;
   const unsigned long long cap_chunks = prep_chunk_bound_per_row(O, n) * (unsigned long long)I;
   const size_t sz_lst = align_up((size_t)I * P * 16, 256);
-  const size_t sz_dense = align_up((size_t)I * dstride * 2, 256);
+  const size_t sz_dense = align_up((size_t)I * dstride * esz, 256);
   const size_t sz_probe = align_up((size_t)I * kP * 2, 256);
-  const size_t sz_tables = sz_lst + sz_dense + sz_probe + 256;
-  const size_t sz_tmp = align_up((size_t)cap_chunks * kCS * 3 + (size_t)cap_chunks * 2, 256);
+  const size_t sz_scale = (wk == kWeightQ8) ? align_up((size_t)I * 2, 256) : 0;
+  const size_t sz_tables = sz_lst + sz_dense + sz_probe + sz_scale + 256;
+  const size_t sz_tmp = align_up((size_t)cap_chunks * kCS * (esz + 1) + (size_t)cap_chunks * 2, 256);
   if (!within_cap(sz_tables + sz_tmp)) return EFFORT_ERR_NOMEM;
   if (cap_chunks >= (1ull << 31)) return EFFORT_ERR_UNSUPPORTED;
 
@@ -310,6 +316,7 @@ effort_status_t effort_prepare(const void* W, int64_t in_dim, int64_t out_dim, f
   d.n = n;
   d.P = P;
   d.dstride = dstride;
+  d.wk = wk;
   d.kept_total = (unsigned long long)I * (unsigned long long)n;
   int prank[kP];
   for (int k = 1; k <= kP; ++k) {
@@ -333,19 +340,25 @@ effort_status_t effort_prepare(const void* W, int64_t in_dim, int64_t out_dim, f
   if ((st = tmp.alloc(sz_tmp)) != EFFORT_OK) return fail(st);
   char* tb = (char*)h->tables.p;
   d.lst = (const uint4*)tb;
-  d.wdense = (const uint16_t*)(tb + sz_lst);
+  void* dense = tb + sz_lst;
+  if (wk == kWeightQ8) d.wdense8 = (const int8_t*)dense;
+  else d.wdense = (const uint16_t*)dense;
   d.probes = (const uint16_t*)(tb + sz_lst + sz_dense);
-  unsigned* ctl = (unsigned*)(tb + sz_lst + sz_dense + sz_probe);  // [0] chunk counter, [1] max |w| bits, [2] status
-  uint16_t* tvals = (uint16_t*)tmp.p;
-  uint8_t* tgaps = (uint8_t*)(tvals + (size_t)cap_chunks * kCS);
+  if (wk == kWeightQ8) d.scales = (const uint16_t*)(tb + sz_lst + sz_dense + sz_probe);
+  unsigned* ctl = (unsigned*)(tb + sz_lst + sz_dense + sz_probe + sz_scale);  // [0] chunks, [1] max |w|, [2] status
+  void* tvals = tmp.p;
+  uint8_t* tgaps = (uint8_t*)tmp.p + (size_t)cap_chunks * kCS * esz;
   uint16_t* thead = (uint16_t*)(tgaps + (size_t)cap_chunks * kCS);
 
   cudaStream_t s = (cudaStream_t)stream;
   h->last_stream = s;
   cudaError_t e = cudaMemsetAsync(h->tables.p, 0, sz_tables, s);
+  // the handle keeps its own copy of the row scales
+  if (e == cudaSuccess && wk == kWeightQ8)
+    e = cudaMemcpyAsync((void*)d.scales, scales, (size_t)I * 2, cudaMemcpyDefault, s);
   if (e == cudaSuccess)
-    e = launch_prep((const uint16_t*)W, I, O, n, P, dstride, prank, (uint16_t*)d.wdense, (uint16_t*)d.probes, tvals,
-                    tgaps, thead, (uint4*)d.lst, ctl, (unsigned)cap_chunks, ctl + 2, s);
+    e = launch_prep(W, d.scales, wk, I, O, n, P, dstride, prank, dense, (uint16_t*)d.probes, tvals, tgaps, thead,
+                    (uint4*)d.lst, ctl, (unsigned)cap_chunks, ctl + 2, s);
   unsigned ctl_h[3] = {0, 0, 0};
   if (e == cudaSuccess) e = cudaMemcpyAsync(ctl_h, ctl, 12, cudaMemcpyDeviceToHost, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
@@ -357,13 +370,14 @@ effort_status_t effort_prepare(const void* W, int64_t in_dim, int64_t out_dim, f
   // the used chunks into storage of the exact size
   const size_t nch = ctl_h[0];
   d.total_chunks = (unsigned)nch;
-  const size_t cv = align_up(nch * kCS * 2, 256), cg = align_up(nch * kCS, 256), chd = align_up(nch * 2 + 2, 256);
+  const size_t cv = align_up(nch * kCS * esz, 256), cg = align_up(nch * kCS, 256), chd = align_up(nch * 2 + 2, 256);
   if ((st = h->chunks.alloc(cv + cg + chd)) != EFFORT_OK) return fail(st);
   char* cb = (char*)h->chunks.p;
-  d.vals = (const uint16_t*)cb;
+  if (wk == kWeightQ8) d.vals8 = (const int8_t*)cb;
+  else d.vals = (const uint16_t*)cb;
   d.gaps = (const uint8_t*)(cb + cv);
   d.head = (const uint16_t*)(cb + cv + cg);
-  e = cudaMemcpyAsync((void*)d.vals, tvals, nch * kCS * 2, cudaMemcpyDeviceToDevice, s);
+  e = cudaMemcpyAsync(cb, tvals, nch * kCS * esz, cudaMemcpyDeviceToDevice, s);
   if (e == cudaSuccess) e = cudaMemcpyAsync((void*)d.gaps, tgaps, nch * kCS, cudaMemcpyDeviceToDevice, s);
   if (e == cudaSuccess) e = cudaMemcpyAsync((void*)d.head, thead, nch * 2, cudaMemcpyDeviceToDevice, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
@@ -378,6 +392,16 @@ effort_status_t effort_prepare(const void* W, int64_t in_dim, int64_t out_dim, f
   if ((st = h->stage.alloc(stage_out_offset(I) + (size_t)O * 4)) != EFFORT_OK) return fail(st);
   *out_handle = h;
   return EFFORT_OK;
+}
+
+effort_status_t effort_prepare(const void* W, int64_t in_dim, int64_t out_dim, float keep_fraction, void* stream,
+                               effort_handle_t* out_handle) {
+  return prepare_impl(W, nullptr, kWeightF16, in_dim, out_dim, keep_fraction, stream, out_handle);
+}
+
+effort_status_t effort_prepare_q8(const int8_t* q, const uint16_t* scales, int64_t in_dim, int64_t out_dim,
+                                  float keep_fraction, void* stream, effort_handle_t* out_handle) {
+  return prepare_impl(q, scales, kWeightQ8, in_dim, out_dim, keep_fraction, stream, out_handle);
 }
 
 effort_status_t effort_gemv_ex(effort_handle_t h, const void* v, effort_dtype_t v_dtype, float effort, float* out,
@@ -696,13 +720,16 @@ effort_status_t effort_get_layout(effort_handle_t h, effort_layout_t* L) {
   L->n_probes = kP;
   L->dense_stride = h->hd.dstride;
   L->total_chunks = h->hd.total_chunks;
-  L->vals = h->hd.vals;
+  const bool q8 = h->hd.wk == kWeightQ8;
+  L->vals = q8 ? (const void*)h->hd.vals8 : (const void*)h->hd.vals;
   L->gaps = h->hd.gaps;
   L->head = h->hd.head;
   L->lists = h->hd.lst;
-  L->wdense = h->hd.wdense;
+  L->wdense = q8 ? (const void*)h->hd.wdense8 : (const void*)h->hd.wdense;
   L->probes = h->hd.probes;
   L->scratch_bytes = h->ws.bytes;
+  L->weight_kind = h->hd.wk;
+  L->scales = h->hd.scales;
   return EFFORT_OK;
 }
 

@@ -104,6 +104,41 @@ __device__ __forceinline__ unsigned tau_of(float a, float x) {
   return lo;
 }
 
+// Q8: the smallest |q| m (0..128) with fl32(a * (s m)) >= x, as the binary16
+// bits of m; 0x7C00 if none.  s m is exact in fp32 (11 + 8 significant
+// bits), so the test is the oracle's fl32(|v_i| |w_ij|) >= c; it does not
+// decrease as m grows, so a binary search finds the first m that passes.
+__device__ __forceinline__ unsigned tau_q8(float a, float s, float x) {
+  if (!(x > 0.0f)) return 0u;
+  if (!(__fmul_rn(a, __fmul_rn(s, 128.0f)) >= x)) return 0x7C00u;
+  int lo = 0, hi = 128;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (__fmul_rn(a, __fmul_rn(s, (float)mid)) >= x) hi = mid;
+    else lo = mid + 1;
+  }
+  return __half_as_ushort(__int2half_rn(lo));
+}
+
+// Q8: 8 int8 values (two words) as four words of two binary16 values each
+// (every int8 is a binary16 value), in the order of the fp16 layout.  Each
+// byte is biased to u = q + 128 (an xor of its top bit) and placed under the
+// high byte 0x64: the binary16 with bits 0x64uu is 1024 + u, so one packed
+// subtraction of 1152 gives q exactly.
+__device__ __forceinline__ uint4 widen_q8(unsigned lo, unsigned hi) {
+  const unsigned a = lo ^ 0x80808080u, b = hi ^ 0x80808080u;
+  const __half2 bias = __halves2half2(__ushort_as_half((unsigned short)0x6480u),
+                                      __ushort_as_half((unsigned short)0x6480u));  // 1152
+  unsigned o[4] = {__byte_perm(a, 0x64646464u, 0x5140u), __byte_perm(a, 0x64646464u, 0x5342u),
+                   __byte_perm(b, 0x64646464u, 0x5140u), __byte_perm(b, 0x64646464u, 0x5342u)};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const __half2 h = __hsub2(*reinterpret_cast<const __half2*>(&o[k]), bias);
+    o[k] = *reinterpret_cast<const unsigned*>(&h);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
 // Debug builds (-DEFFORT_DEBUG) check every index a kernel takes from data
 // (rows, chunks, decoded columns, stage offsets) before using it; a bad one
 // sets kStatusInternal (effort_check then returns EFFORT_ERR_DEVICE) and the
@@ -239,6 +274,8 @@ struct KSmem {
   unsigned* cidx;
   unsigned short* cunit;
   unsigned* ctl;
+  float* us;      // Q8: scale of each unit's row
+  float* cscale;  // Q8: |scale| of each cutoff row
 };
 
 // Stored chunks of a list whose first magnitude reaches tau: the first 16
@@ -262,8 +299,12 @@ __device__ __forceinline__ unsigned chunks_reaching(const HandleDesc& hd, const 
 // V vectors per launch (1, or 2 on one matrix: the union of their prefixes is
 // read once and each vector's threshold applied to it).  Per-vector state is
 // held in arrays of V.
-template <int V>
+// WK: kWeightF16, or kWeightQ8 (int8 values widened to binary16 as they are
+// loaded, so the masks and products below serve both; the row scale enters
+// the chart, the thresholds and the unit's v).
+template <int V, int WK>
 __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ Job jb) {
+  constexpr bool kQ8 = WK == kWeightQ8;
   extern __shared__ __align__(128) unsigned char smem[];
   const HandleDesc& hd = jb.hd;
   const WsPtrs& ws = jb.ws;  // vector 0's scratch holds the grid barrier and the call's counters
@@ -281,7 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ 
   const int nu = (j0 < I) ? (I - 1 - j0) / nbp + 1 : 0;
   const int pwid = min(kPW, O - p * kPW);
   const int stripes = (pwid + kStripe - 1) / kStripe;
-  const unsigned dense_bytes = (unsigned)stripes * (kStripe * 2);
+  const unsigned dense_bytes = (unsigned)stripes * (kStripe * (kQ8 ? 1 : 2));
   const int mode = jb.mode;
 
   // per-vector arguments
@@ -322,6 +363,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ 
   S.cidx = reinterpret_cast<unsigned*>(smem + L.cidx);
   S.cunit = reinterpret_cast<unsigned short*>(smem + L.cunit);
   S.ctl = reinterpret_cast<unsigned*>(smem + L.ctl);
+  S.us = reinterpret_cast<float*>(smem + L.us);
+  S.cscale = reinterpret_cast<float*>(smem + L.cscale);
   unsigned* wsum = S.ctl + kCtlWsum;
   unsigned* status = ws.hdr + kHdrStatus;
   const int chs = nr * kP;  // chart entries of one vector (the chart of vector k at S.chart + k rp kP)
@@ -343,7 +386,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ 
   if (mode == kModeAll) {
     // every unit is read whole from the dense copy: ask L2 for them now
     for (int u = tid; u < nu0; u += kThreads)
-      prefetch_l2_bulk(hd.wdense + (size_t)(j0 + u * nbp) * hd.dstride + (size_t)p * kPW, dense_bytes);
+      if constexpr (kQ8)
+        prefetch_l2_bulk(hd.wdense8 + (size_t)(j0 + u * nbp) * hd.dstride + (size_t)p * kPW, dense_bytes);
+      else
+        prefetch_l2_bulk(hd.wdense + (size_t)(j0 + u * nbp) * hd.dstride + (size_t)p * kPW, dense_bytes);
   }
   __syncthreads();
 
@@ -390,6 +436,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ 
     for (int u = tid; u < nu0; u += kThreads) {
       const int i = j0 + u * nbp;
       S.uv[k * kUnitCap + u] = jb.vdtype ? __half2float(vh[i]) : vf[i];
+      if constexpr (kQ8)
+        if (k == 0) S.us[u] = h2f(hd.scales[i]);
     }
     for (int t0 = 0; t0 < nr; t0 += kThreads) {
       const int t = t0 + tid;
@@ -399,6 +447,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ 
         if (!isfinite(x)) atomicOr(status, kStatusNonfiniteV);
         ax = fabsf(x);
         S.absv[k * rp + t] = ax;
+        if constexpr (kQ8)
+          if (k == 0) S.cscale[t] = fabsf(h2f(hd.scales[r0 + t]));
         if (k == 0 && jb.rowlen_out) jb.rowlen_out[r0 + t] = (mode == kModeAll) ? (unsigned)hd.n : 0u;
       }
 #pragma unroll
@@ -427,7 +477,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ 
         const unsigned pb = S.chart[e];  // probe bits, replaced by vector 0's chart
 #pragma unroll
         for (int k = V - 1; k >= 0; --k) {
-          const unsigned xb = __float_as_uint(__fmul_rn(S.absv[k * rp + (e >> 4)], h2f(pb)));
+          const float pm = kQ8 ? __fmul_rn(S.cscale[e >> 4], h2f(pb)) : h2f(pb);  // probe |w| (exact)
+          const unsigned xb = __float_as_uint(__fmul_rn(S.absv[k * rp + (e >> 4)], pm));
           S.chart[k * rp * kP + e] = xb;
           atomicAdd(&S.hist[k * kBins0 + (xb >> 19)], w);
           rank[k * chs + e] = (unsigned short)atomicAdd(&hcnt[k * kBins0 + (xb >> 19)], 1u);
@@ -438,7 +489,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ 
         const unsigned pb = S.chart[e];
 #pragma unroll
         for (int k = V - 1; k >= 0; --k)
-          S.chart[k * rp * kP + e] = __float_as_uint(__fmul_rn(S.absv[k * rp + (e >> 4)], h2f(pb)));
+          S.chart[k * rp * kP + e] = __float_as_uint(
+              __fmul_rn(S.absv[k * rp + (e >> 4)], kQ8 ? __fmul_rn(S.cscale[e >> 4], h2f(pb)) : h2f(pb)));
       }
     __syncthreads();
     // each bin's first slot in the block's segment (bins in ascending order)
@@ -665,7 +717,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ 
   for (int k = 0; k < V; ++k) {
     sc[k] = 1.0f;
     inv_sc[k] = 1.0f;
-    const float bound = 2.0f * __uint_as_float(vsum_bits[k]) * h2f(hd.wmax_bits);
+    const float bound = 2.0f * __uint_as_float(vsum_bits[k]) * (kQ8 ? __uint_as_float(hd.wmax_bits) : h2f(hd.wmax_bits));
     if (bound > 0.0f && isfinite(bound)) {
       int ex = 0;
       frexpf(bound, &ex);  // bound < 2^ex
@@ -711,6 +763,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ 
         for (int u = tid; u < nuR; u += kThreads) {
           const int i = j0 + (u0 + u) * nbp;
           S.uv[k * kUnitCap + u] = jb.vdtype ? __half2float(vh[i]) : vf[i];
+          if constexpr (kQ8)
+            if (k == 0) S.us[u] = h2f(hd.scales[i]);
         }
       }
       if (tid == 0) S.ctl[kCtlExtraDense] = 0u;
@@ -732,10 +786,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ 
         if (count_all[k]) {
           all = true;
         } else {
-          tau = tau_of(fabsf(S.uv[k * kUnitCap + u]), c[k]);
+          if constexpr (kQ8)
+            tau = tau_q8(fabsf(S.uv[k * kUnitCap + u]), fabsf(S.us[u]), c[k]);
+          else
+            tau = tau_of(fabsf(S.uv[k * kUnitCap + u]), c[k]);
           tmin = min(tmin, tau);
         }
         S.utau[k * kUnitCap + u] = tau;
+        if constexpr (kQ8) S.uv[k * kUnitCap + u] = __fmul_rn(S.uv[k * kUnitCap + u], S.us[u]);  // v_i s_i
       }
       if (all) {
         kind = 1;
@@ -777,7 +835,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ 
     const unsigned nch = S.ctl[kCtlChunks];
     if (tid == 0) {
       planned_dense += (unsigned long long)nd * dense_bytes;
-      planned_sparse += (unsigned long long)nch * (unsigned)(kCS * 3);
+      planned_sparse += (unsigned long long)nch * (unsigned)(kCS * (kQ8 ? 2 : 3));
     }
     EFFORT_MARK(7);
 
@@ -785,7 +843,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ 
     // half + 2, ... of the dense list, kDenseBatch loads in flight per lane
     if constexpr (V == 1) {
       if (sj < stripes) {
-        const uint16_t* base = hd.wdense + (size_t)p * kPW + sj * kStripe + 8 * lane;
+        const size_t lane_off = (size_t)p * kPW + sj * kStripe + 8 * lane;
+        const uint16_t* base = hd.wdense + lane_off;
+        const int8_t* base8 = hd.wdense8 + lane_off;
         for (unsigned k0 = (unsigned)half; k0 < nd; k0 += 2 * kDenseBatch) {
           uint4 wv[kDenseBatch];
           unsigned tq[kDenseBatch];
@@ -801,7 +861,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ 
             if (k < nd) {
               const unsigned uu = S.dlist[k];
               const int i = j0 + (u0 + (int)uu) * nbp;
-              wv[q] = __ldcs(reinterpret_cast<const uint4*>(base + (size_t)i * hd.dstride));
+              if constexpr (kQ8) {
+                const uint2 r = __ldcs(reinterpret_cast<const uint2*>(base8 + (size_t)i * hd.dstride));
+                wv[q].x = r.x;
+                wv[q].y = r.y;
+              } else {
+                wv[q] = __ldcs(reinterpret_cast<const uint4*>(base + (size_t)i * hd.dstride));
+              }
               tq[q] = S.utau[uu];
               vq[q] = S.uv[uu];
               iq[q] = i;
@@ -811,6 +877,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ 
           for (int q = 0; q < kDenseBatch; ++q) {
             const unsigned tau2 = tq[q] | (tq[q] << 16);
             const float2 v2 = make_float2(vq[q], vq[q]);
+            if constexpr (kQ8) wv[q] = widen_q8(wv[q].x, wv[q].y);
             const unsigned w4[4] = {wv[q].x, wv[q].y, wv[q].z, wv[q].w};
             unsigned rc = 0;
 #pragma unroll
@@ -834,7 +901,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ 
     } else {
       // two vectors: one load of each unit, each vector's mask and FMA
     if (sj < stripes) {
-      const uint16_t* base = hd.wdense + (size_t)p * kPW + sj * kStripe + 8 * lane;
+      const size_t lane_off = (size_t)p * kPW + sj * kStripe + 8 * lane;
+      const uint16_t* base = hd.wdense + lane_off;
+      const int8_t* base8 = hd.wdense8 + lane_off;
       for (unsigned k0 = (unsigned)half; k0 < nd; k0 += 2 * kDenseBatch) {
         uint4 wv[kDenseBatch];
         unsigned uq[kDenseBatch];
@@ -845,12 +914,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ 
           uq[q] = 0xFFFFu;
           if (k < nd) {
             uq[q] = S.dlist[k];
-            wv[q] = __ldcs(reinterpret_cast<const uint4*>(base + (size_t)(j0 + (u0 + (int)uq[q]) * nbp) * hd.dstride));
+            const size_t roff = (size_t)(j0 + (u0 + (int)uq[q]) * nbp) * hd.dstride;
+            if constexpr (kQ8) {
+              const uint2 r = __ldcs(reinterpret_cast<const uint2*>(base8 + roff));
+              wv[q].x = r.x;
+              wv[q].y = r.y;
+            } else {
+              wv[q] = __ldcs(reinterpret_cast<const uint4*>(base + roff));
+            }
           }
         }
 #pragma unroll
         for (int q = 0; q < kDenseBatch; ++q) {
           const bool okq = uq[q] != 0xFFFFu;
+          if constexpr (kQ8) wv[q] = widen_q8(wv[q].x, wv[q].y);
           const unsigned w4[4] = {wv[q].x, wv[q].y, wv[q].z, wv[q].w};
 #pragma unroll
           for (int k = 0; k < V; ++k) {
@@ -897,7 +974,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ 
           const unsigned ci = S.cidx[t];
           if (EFFORT_IN_RANGE(ci < hd.total_chunks, status)) {
             uq[q] = S.cunit[t];
-            vv[q] = __ldcs(reinterpret_cast<const uint4*>(hd.vals + (size_t)ci * kCS) + sl);
+            if constexpr (kQ8) {
+              const uint2 r = __ldcs(reinterpret_cast<const uint2*>(hd.vals8 + (size_t)ci * kCS) + sl);
+              vv[q].x = r.x;
+              vv[q].y = r.y;
+            } else {
+              vv[q] = __ldcs(reinterpret_cast<const uint4*>(hd.vals + (size_t)ci * kCS) + sl);
+            }
             gg[q] = __ldcs(reinterpret_cast<const uint2*>(hd.gaps + (size_t)ci * kCS) + sl);
           }
         }
@@ -922,6 +1005,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ 
           if (sl >= o) ex += y;
         }
         const int basecol = ex - cs[7] - 1;
+        if constexpr (kQ8) vv[q] = widen_q8(vv[q].x, vv[q].y);
         const unsigned w4[4] = {vv[q].x, vv[q].y, vv[q].z, vv[q].w};
 #pragma unroll
         for (int k = 0; k < V; ++k) {
@@ -1076,8 +1160,13 @@ cudaError_t effort_kernel_attributes(int I, size_t smem) {
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
   if (e != cudaSuccess) return e;
   if ((size_t)optin < smem) return cudaErrorInvalidValue;
-  e = cudaFuncSetAttribute(k_effort<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
-  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_effort<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+  e = cudaFuncSetAttribute(k_effort<1, kWeightF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k_effort<2, kWeightF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k_effort<1, kWeightQ8>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k_effort<2, kWeightQ8>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
   return e;
 }
 
@@ -1085,11 +1174,17 @@ cudaError_t effort_kernel_attributes(int I, size_t smem) {
 int effort_grid_size(int I, int sms, size_t smem) {
   (void)I;
   int nbk = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nbk, k_effort<2>, kThreads, smem) != cudaSuccess) {
-    cudaGetLastError();
-    return 0;
+  // every instantiation must fit one block per SM
+  const void* fns[4] = {(const void*)k_effort<1, kWeightF16>, (const void*)k_effort<2, kWeightF16>,
+                        (const void*)k_effort<1, kWeightQ8>, (const void*)k_effort<2, kWeightQ8>};
+  for (const void* f : fns) {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nbk, f, kThreads, smem) != cudaSuccess) {
+      cudaGetLastError();
+      return 0;
+    }
+    if (nbk < 1) return 0;
   }
-  return nbk >= 1 ? sms : 0;
+  return sms;
 }
 
 // One matvec (nvec = 1) or two on one matrix (nvec = 2, job.v2 ...).  smem is
@@ -1106,7 +1201,11 @@ cudaError_t launch_effort(const Job& job, int nb, size_t smem, cudaStream_t stre
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return nvec == 2 ? cudaLaunchKernelEx(&cfg, k_effort<2>, job) : cudaLaunchKernelEx(&cfg, k_effort<1>, job);
+  if (job.hd.wk == kWeightQ8)
+    return nvec == 2 ? cudaLaunchKernelEx(&cfg, k_effort<2, kWeightQ8>, job)
+                     : cudaLaunchKernelEx(&cfg, k_effort<1, kWeightQ8>, job);
+  return nvec == 2 ? cudaLaunchKernelEx(&cfg, k_effort<2, kWeightF16>, job)
+                   : cudaLaunchKernelEx(&cfg, k_effort<1, kWeightF16>, job);
 }
 
 }  // namespace effort

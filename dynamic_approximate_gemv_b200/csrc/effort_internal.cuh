@@ -25,6 +25,11 @@
 //   * probes: [I][16] |w| bits at the midpoint ranks of 16 equal segments of
 //     the kept list (the `get_probes` step of the pages' pseudo-code).
 //   * wmax_bits: the largest kept |w| (bounds every partial sum of a call).
+//
+// Q8 matrices (int8 q and one binary16 scale s_i per row, w = s_i q) use the
+// same layout with int8 values (vals8, wdense8) and the row scales; heads,
+// tails and probes hold the binary16 bits of |q| (0 on a zero-scale row),
+// and wmax_bits the fp32 bits of the largest |s_i| |q|.
 #pragma once
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -53,6 +58,9 @@ constexpr int kDenseThreads = 256;
 constexpr int kDenseRowsPerItem = 8;  // dense rows a warp accumulates per stripe item
 constexpr int kMaxPanels = 16;        // 32768 / 2048
 
+// weight kinds of a prepared matrix
+enum : int { kWeightF16 = 0, kWeightQ8 = 1 };
+
 // call modes decided on the host from K and the kept count
 enum : int { kModeSelect = 0, kModeAll = 1, kModeNone = 2 };
 // device status bits
@@ -79,7 +87,11 @@ struct HandleDesc {
   const uint16_t* probes;  // [I][kP]
   int I, O, n, P, dstride;
   unsigned total_chunks;
-  unsigned wmax_bits;      // binary16 bits of the largest kept |w|
+  unsigned wmax_bits;      // binary16 bits of the largest kept |w| (Q8: fp32 bits)
+  int wk;                  // kWeightF16 or kWeightQ8
+  const int8_t* vals8;     // Q8: [total chunks * kCS] (vals is null)
+  const int8_t* wdense8;   // Q8: [I][dstride] (wdense is null)
+  const uint16_t* scales;  // Q8: [I] binary16 row scales
   unsigned long long kept_total;
   int pw[kP];              // probe weights (entries each probe stands for)
 };
@@ -136,7 +148,7 @@ __host__ __device__ inline int rows_per_block(int I, int nb) { return (I + nb - 
 // Shared memory of the matvec kernel (byte offsets) for V vectors per launch
 // (V = 2: two vectors on one matrix read the union of their prefixes once).
 struct SmemLayout {
-  size_t iacc, chart, absv, hist, hist2, cand, ulst, uhead, uv, utau, dlist, cidx, cunit, ctl, total;
+  size_t iacc, chart, absv, hist, hist2, cand, ulst, uhead, uv, utau, dlist, cidx, cunit, ctl, us, cscale, total;
 };
 __host__ __device__ inline SmemLayout smem_layout(int I, int nb, int V = 1) {
   SmemLayout L;
@@ -163,6 +175,8 @@ __host__ __device__ inline SmemLayout smem_layout(int I, int nb, int V = 1) {
   L.cunit = take((size_t)kChunkCap * 2);              // and the unit of each (before the dispatch: the
                                                       // crossing-bin gather's per-block offsets)
   L.ctl = take(256 * 4);                              // control words
+  L.us = take((size_t)kUnitCap * 4);                  // Q8: scale of the unit's row
+  L.cscale = take(rp * 4);                            // Q8: |scale| of the cutoff rows
   L.total = o;
   return L;
 }

@@ -20,6 +20,12 @@
 //      The greedy cut takes as many ranks as fit in 64 slots.  Chunks are
 //      placed through a global counter; the host then copies the used part
 //      into storage of the exact size.
+//
+// Q8 weights (int8 q and a binary16 scale s_i per row, w = s_i q exactly)
+// take the same steps: the sort key holds the binary16 bits of |q| (0 for a
+// row whose scale is 0, where every |w| is 0), so lists, chunks, heads,
+// tails and probes come out as for fp16 weights of magnitude |q|; the
+// values (dense copy and chunk slots) are the int8 q.
 #include "effort_internal.cuh"
 
 #define EFFORT_PREP_KEYS_MAX 32768
@@ -28,11 +34,13 @@
 namespace effort {
 
 struct PrepArgs {
-  const uint16_t* W;
+  const void* W;             // [I][O] binary16 bits, or int8 (Q8)
+  const uint16_t* scales;    // Q8: [I] binary16 row scales; null for fp16
+  int wk;                    // kWeightF16 or kWeightQ8
   int I, O, n, P, dstride, Np;
-  uint16_t* wdense;
+  void* wdense;              // [I][dstride] of the weight type
   uint16_t* probes;
-  uint16_t* vals;        // capacity cap_chunks * kCS
+  void* vals;                // capacity cap_chunks * kCS, of the weight type
   uint8_t* gaps;         // capacity cap_chunks * kCS
   uint16_t* head;        // capacity cap_chunks
   uint4* lst;            // [I][P]
@@ -113,23 +121,45 @@ __device__ __forceinline__ int chunk_slots(const uint32_t* list, int q, int t, i
   return t + warp_sum(f0 + f1);
 }
 
+// Chunk slot `slot` gets the weight at column j of the row (or +0 when the
+// row pointers are null: fillers and pads).
+__device__ __forceinline__ void put_val(const PrepArgs& a, size_t slot, const uint16_t* row, const int8_t* row8, int j) {
+  if (a.wk == kWeightQ8) static_cast<int8_t*>(a.vals)[slot] = row8 ? row8[j] : (int8_t)0;
+  else static_cast<uint16_t*>(a.vals)[slot] = row ? row[j] : (uint16_t)0;
+}
+
 __global__ void __launch_bounds__(kPrepThreads, 1) k_prep_rows(const __grid_constant__ PrepArgs a) {
   extern __shared__ uint32_t keys[];  // Np keys, then the per-warp list buffers
   __shared__ int panel_n[kMaxPanels];
   const int O = a.O, n = a.n, P = a.P;
   const int i = blockIdx.x;
-  const uint16_t* row = a.W + (size_t)i * O;
+  const bool q8 = a.wk == kWeightQ8;
+  const uint16_t* row = q8 ? nullptr : static_cast<const uint16_t*>(a.W) + (size_t)i * O;
+  const int8_t* row8 = q8 ? static_cast<const int8_t*>(a.W) + (size_t)i * O : nullptr;
   uint32_t* lists = keys + a.Np;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 
   if (threadIdx.x < kMaxPanels) panel_n[threadIdx.x] = 0;
   bool bad = false;
+  unsigned sbits = 0;
+  if (q8) {
+    sbits = a.scales[i];
+    if ((sbits & 0x7C00u) == 0x7C00u) bad = true;
+  }
+  const bool szero = q8 && (sbits & 0x7FFFu) == 0u;
   for (int j = threadIdx.x; j < a.Np; j += blockDim.x) {
     uint32_t key = 0xFFFFFFFFu;
     if (j < O) {
-      const uint32_t b = row[j];
-      if ((b & 0x7C00u) == 0x7C00u) bad = true;
-      key = ((0x7FFFu - (b & 0x7FFFu)) << 16) | (uint32_t)j;
+      uint32_t mag;
+      if (q8) {
+        // |q| as binary16 bits (exact for 0..128); every |w| of a zero-scale row is 0
+        mag = szero ? 0u : (uint32_t)__half_as_ushort(__int2half_rn(abs((int)row8[j])));
+      } else {
+        const uint32_t b = row[j];
+        if ((b & 0x7C00u) == 0x7C00u) bad = true;
+        mag = b & 0x7FFFu;
+      }
+      key = ((0x7FFFu - mag) << 16) | (uint32_t)j;
     }
     keys[j] = key;
   }
@@ -140,10 +170,18 @@ __global__ void __launch_bounds__(kPrepThreads, 1) k_prep_rows(const __grid_cons
   // dense copy of the kept weights (dropped ones stay +0.0 from the memset)
   for (int r = threadIdx.x; r < n; r += blockDim.x) {
     const int j = (int)(keys[r] & 0xFFFFu);
-    a.wdense[(size_t)i * a.dstride + j] = row[j];
+    if (q8) static_cast<int8_t*>(a.wdense)[(size_t)i * a.dstride + j] = row8[j];
+    else static_cast<uint16_t*>(a.wdense)[(size_t)i * a.dstride + j] = row[j];
     atomicAdd(&panel_n[j / kPW], 1);
   }
-  if (threadIdx.x == 0) atomicMax(a.chunk_count + 1, 0x7FFFu - (keys[0] >> 16));
+  // the largest kept |w|: binary16 bits (fp16), or fp32 bits of |s_i| max |q| (Q8, exact)
+  if (threadIdx.x == 0) {
+    const unsigned m = 0x7FFFu - (keys[0] >> 16);
+    atomicMax(a.chunk_count + 1,
+              q8 ? __float_as_uint(fabsf(__half2float(__ushort_as_half((unsigned short)sbits))) *
+                                   __half2float(__ushort_as_half((unsigned short)m)))
+                 : m);
+  }
   if (threadIdx.x < kP) {
     const int r = a.prank[threadIdx.x];
     a.probes[(size_t)i * kP + threadIdx.x] = (r >= 0) ? (uint16_t)(0x7FFFu - (keys[r] >> 16)) : (uint16_t)0;
@@ -220,23 +258,23 @@ __global__ void __launch_bounds__(kPrepThreads, 1) k_prep_rows(const __grid_cons
       if (lane < t) {
         const int e = x0 - inc0;  // first slot of this entry's fillers
         for (int f = 0; f < f0; ++f) {
-          a.vals[slot0 + e + f] = 0;
+          put_val(a, slot0 + e + f, nullptr, nullptr, 0);
           a.gaps[slot0 + e + f] = 255;
         }
-        a.vals[slot0 + e + f0] = row[pbase + (int)s0];
+        put_val(a, slot0 + e + f0, row, row8, pbase + (int)s0);
         a.gaps[slot0 + e + f0] = (uint8_t)(g0 - 255 * f0);
       }
       if (lane + 32 < t) {
         const int e = x1 - inc1;
         for (int f = 0; f < f1; ++f) {
-          a.vals[slot0 + e + f] = 0;
+          put_val(a, slot0 + e + f, nullptr, nullptr, 0);
           a.gaps[slot0 + e + f] = 255;
         }
-        a.vals[slot0 + e + f1] = row[pbase + (int)s1];
+        put_val(a, slot0 + e + f1, row, row8, pbase + (int)s1);
         a.gaps[slot0 + e + f1] = (uint8_t)(g1 - 255 * f1);
       }
       for (int z = used + lane; z < kCS; z += 32) {
-        a.vals[slot0 + z] = 0;
+        put_val(a, slot0 + z, nullptr, nullptr, 0);
         a.gaps[slot0 + z] = 0;
       }
       if (lane == 0) a.head[base + k] = (uint16_t)(0x7FFFu - (list[q] >> 16));
@@ -255,11 +293,13 @@ cudaError_t prep_attributes() {
                               (int)prep_smem_bytes(EFFORT_PREP_KEYS_MAX));
 }
 
-cudaError_t launch_prep(const uint16_t* W, int I, int O, int n, int P, int dstride, const int* prank,
-                        uint16_t* wdense, uint16_t* probes, uint16_t* vals, uint8_t* gaps, uint16_t* head, uint4* lst,
-                        unsigned* chunk_count, unsigned cap_chunks, unsigned* status, cudaStream_t stream) {
+cudaError_t launch_prep(const void* W, const uint16_t* scales, int wk, int I, int O, int n, int P, int dstride,
+                        const int* prank, void* wdense, uint16_t* probes, void* vals, uint8_t* gaps, uint16_t* head,
+                        uint4* lst, unsigned* chunk_count, unsigned cap_chunks, unsigned* status, cudaStream_t stream) {
   PrepArgs a;
   a.W = W;
+  a.scales = scales;
+  a.wk = wk;
   a.I = I;
   a.O = O;
   a.n = n;

@@ -82,6 +82,29 @@ effort_status_t effort_prepare(const void* W, int64_t in_dim, int64_t out_dim, f
                                void* stream, effort_handle_t* out_handle);
 
 /*
+ * effort_prepare_q8 -- effort_prepare for Q8 weights: int8 values q and one
+ *   binary16 scale per row, the weight being w_ij = s_i * q_ij, taken exactly
+ *   (the post says Q8 is in the works and the author that the algorithm
+ *   should work on top of Q8: Hacker News item 40067677, "Show HN: Speeding
+ *   up LLM inference 2x times (possibly)", the post text and the author's
+ *   replies).  Everything the matvec computes follows from those weights as
+ *   for effort_prepare: row order |w| descending with ties to the lower
+ *   column, keep, probes, the cutoff c, the used set fl32(|v_i| |w_ij|) >= c
+ *   and out.  The stored matrix holds q as int8: 2 bytes per chunk slot
+ *   (value and gap) and 1 byte per column of the dense copy.
+ *   q: device int8 [in_dim x out_dim], row-major (row i multiplies v[i]);
+ *   scales: device binary16 bits [in_dim], 2-byte aligned, finite (zero and
+ *   negative scales are allowed); both are read during the call only (the
+ *   handle keeps its own copy of the scales).
+ *   keep_fraction, stream, out_handle and the limits: as for effort_prepare.
+ *   Returns EFFORT_ERR_NONFINITE if a scale is inf or NaN, EFFORT_ERR_ARG for
+ *   a null or misaligned pointer or a bad keep_fraction.  Every matvec entry
+ *   point accepts the handle (the dense baseline is for binary16 only).
+ */
+effort_status_t effort_prepare_q8(const int8_t* q, const uint16_t* scales, int64_t in_dim, int64_t out_dim,
+                                  float keep_fraction, void* stream, effort_handle_t* out_handle);
+
+/*
  * effort_gemv -- one approximate matvec: `approxMul(v, ...)` of the pages.
  *   v: device fp32 [in_dim]; out: device fp32 [out_dim], fully overwritten.
  *   effort in (0, 1]: K = llround(effort * in_dim * out_dim) products are
@@ -273,6 +296,11 @@ effort_status_t effort_get_info(effort_handle_t h, int64_t* in_dim, int64_t* out
  * wdense: [in_dim][dense_stride] binary16: kept weights at their columns, +0
  *   elsewhere.  probes: [in_dim][16] |w| bits at the probe ranks (0 for empty
  *   segments).  scratch_bytes: the handle's per-call scratch.
+ * weight_kind: 0 for a matrix from effort_prepare, 1 for one from
+ *   effort_prepare_q8.  For Q8, vals and wdense hold int8 q (1 byte per slot
+ *   or column), tail, head and probes hold the binary16 bits of |q| (0 on a
+ *   row whose scale is 0), and scales is the handle's copy of the row
+ *   scales [in_dim] (binary16); null for fp16.
  */
 typedef struct {
   int64_t in_dim, out_dim;
@@ -285,6 +313,8 @@ typedef struct {
   const void* wdense;
   const void* probes;
   size_t scratch_bytes;
+  int32_t weight_kind;
+  const void* scales;
 } effort_layout_t;
 
 effort_status_t effort_get_layout(effort_handle_t h, effort_layout_t* layout);
@@ -296,8 +326,8 @@ effort_status_t effort_destroy(effort_handle_t h);
  * effort_last_call_bytes -- the bytes of the prepared matrix that the handle's
  *   last finished call (effort_gemv, _ex, _host) planned to read: dense_bytes
  *   for the (row, panel) units it read from the dense copy (512 bytes per
- *   256-column stripe), sparse_bytes for the chunks (3 bytes per slot, 64
- *   slots per chunk).  Synchronises the handle's last stream.  The pages have
+ *   256-column stripe; 256 for Q8), sparse_bytes for the chunks (3 bytes per
+ *   slot, 2 for Q8; 64 slots per chunk).  Synchronises the handle's last stream.  The pages have
  *   no counterpart: a measurement service.  dense_bytes, sparse_bytes: host
  *   pointers, non-NULL.
  */

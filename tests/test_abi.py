@@ -26,7 +26,7 @@ def declared_functions():
 
 def test_header_declares_the_boundary():
     names = declared_functions()
-    for must in ("effort_prepare", "effort_gemv", "effort_gemv_ex", "effort_gemv_host", "effort_gemv_batched",
+    for must in ("effort_prepare", "effort_prepare_q8", "effort_gemv", "effort_gemv_ex", "effort_gemv_host", "effort_gemv_batched",
                  "effort_destroy",
                  "effort_dense_gemv", "effort_workspace_create", "effort_status_string"):
         assert must in names
@@ -56,6 +56,14 @@ def test_argument_errors_need_no_device(L):
     assert L.effort_prepare(fake, 4, 40000, ctypes.c_float(1.0), None, ctypes.byref(h)) == 6
     assert L.effort_prepare(fake, 50000, 4, ctypes.c_float(1.0), None, ctypes.byref(h)) == 6
     assert L.effort_prepare(fake, 4, 10, ctypes.c_float(0.04), None, ctypes.byref(h)) == 1  # keeps nothing
+    q8 = L.effort_prepare_q8
+    q8.argtypes = [vp, vp, ctypes.c_int64, ctypes.c_int64, ctypes.c_float, vp, ctypes.POINTER(vp)]
+    assert q8(None, fake, 4, 4, ctypes.c_float(1.0), None, ctypes.byref(h)) == 1      # no q
+    assert q8(vp(0x100001), None, 4, 4, ctypes.c_float(1.0), None, ctypes.byref(h)) == 1  # no scales
+    assert q8(vp(0x100001), vp(0x100001), 4, 4, ctypes.c_float(1.0), None, ctypes.byref(h)) == 1  # odd scales
+    assert q8(vp(0x100001), fake, 4, 4, ctypes.c_float(0.0), None, ctypes.byref(h)) == 1
+    assert q8(vp(0x100001), fake, 4, 40000, ctypes.c_float(1.0), None, ctypes.byref(h)) == 6
+    assert q8(fake, fake, 4, 4, ctypes.c_float(1.0), None, None) == 1
     assert L.effort_gemv(None, fake, ctypes.c_float(0.5), fake, None) == 1
     assert L.effort_gemv_ex(None, fake, 0, ctypes.c_float(0.5), fake, None, None, None, None) == 1
     assert L.effort_gemv_host(None, fake, 0, ctypes.c_float(0.5), fake, None) == 1
