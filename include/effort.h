@@ -13,7 +13,8 @@
  * dispatch and about O(inDim log inDim) for the cutoff.
  *
  * Conventions (all entry points):
- *  - W is [in_dim x out_dim] binary16, row-major: row i holds the weights that
+ *  - W is [in_dim x out_dim] binary16 (or, for effort_prepare_q8, int8 with one
+ *    binary16 scale per row), row-major: row i holds the weights that
  *    multiply v[i], and out[j] = sum_i v[i] * W[i][j] (the matrix is already
  *    "flipped" in the sense of the pages).
  *  - Pointers named W, v, V, out, OUT, *_out are DEVICE pointers unless stated.
