@@ -717,7 +717,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_effort(const __grid_constant__ 
   for (int k = 0; k < V; ++k) {
     sc[k] = 1.0f;
     inv_sc[k] = 1.0f;
-    const float bound = 2.0f * __uint_as_float(vsum_bits[k]) * (kQ8 ? __uint_as_float(hd.wmax_bits) : h2f(hd.wmax_bits));
+    const float wmax = kQ8 ? __uint_as_float(hd.wmax_bits) : h2f(hd.wmax_bits);  // largest kept |w|
+    const float bound = 2.0f * __uint_as_float(vsum_bits[k]) * wmax;
     if (bound > 0.0f && isfinite(bound)) {
       int ex = 0;
       frexpf(bound, &ex);  // bound < 2^ex
