@@ -254,6 +254,18 @@ def read_bytes(in_dim, out_dim, dense, sparse, v_bytes=4):
     return float(dense) + float(sparse) + 2.0 * 16 * in_dim + v_bytes * in_dim + 4.0 * out_dim
 
 
+def algorithmic_bytes_q8(in_dim, out_dim, used, v_bytes=4):
+    """The same for a Q8 matrix: 2 bytes per used product (int8 value and an
+    8-bit position), the probes, one binary16 scale per row, v and out."""
+    return 2.0 * used + 2.0 * 16 * in_dim + 2.0 * in_dim + v_bytes * in_dim + 4.0 * out_dim
+
+
+def read_bytes_q8(in_dim, out_dim, dense, sparse, v_bytes=4):
+    """Planned reads of a Q8 call (int8 dense panel rows, 2-byte chunk slots,
+    as the library reports them) plus probes, row scales, v and out."""
+    return read_bytes(in_dim, out_dim, dense, sparse, v_bytes) + 2.0 * in_dim
+
+
 # ----------------------------------------------------------------- other shapes
 def measure_shape(E, dev, in_dim, out_dim, efforts, dist, n_mats=10, n_vecs=8, seed0=5000, keep=1.0, q8=False):
     """us per matvec and algorithmic GB/s on another workload shape: n_mats
@@ -315,9 +327,8 @@ def measure_shape(E, dev, in_dim, out_dim, efforts, dist, n_mats=10, n_vecs=8, s
         torch.cuda.synchronize()
         us = e0.elapsed_time(e1) * 1000.0 / (reps * steps)
         if q8:
-            # 2 bytes per used product (int8 value and an 8-bit position), probes, row scales, v, out
-            b = algorithmic_bytes(in_dim, out_dim, used) - used + 2.0 * in_dim
-            rb = read_bytes(in_dim, out_dim, dense, sparse) + 2.0 * in_dim
+            b = algorithmic_bytes_q8(in_dim, out_dim, used)
+            rb = read_bytes_q8(in_dim, out_dim, dense, sparse)
             dense_b = 1.0 * in_dim * out_dim + 2.0 * in_dim + 4.0 * in_dim + 4.0 * out_dim
         else:
             b = algorithmic_bytes(in_dim, out_dim, used)

@@ -73,3 +73,15 @@ def test_byte_counts_per_path():
     assert bench.read_bytes(I, O, 2 * I * O, 0) == 2 * I * O + 32 * I + 4 * I + 4 * O
     assert bench.read_bytes(I, O, 10, 20, v_bytes=2) == 30 + 32 * I + 2 * I + 4 * O
     assert bench.read_bytes(I, O, 2 * I * O, 0) < bench.algorithmic_bytes(I, O, I * O)
+
+
+def test_q8_byte_counts():
+    """Q8: 2 bytes per used product, and the row scales (2 bytes per row) on
+    top of the probes, v and out; at effort 1 the planned read is the int8
+    dense copy, half the fp16 one."""
+    import bench
+    I, O = 4096, 14336
+    assert bench.algorithmic_bytes_q8(I, O, 0) == 32 * I + 2 * I + 4 * I + 4 * O
+    assert bench.algorithmic_bytes_q8(I, O, 1000) - bench.algorithmic_bytes_q8(I, O, 0) == 2000
+    assert bench.read_bytes_q8(I, O, I * O, 0) == I * O + 32 * I + 2 * I + 4 * I + 4 * O
+    assert bench.read_bytes_q8(I, O, I * O, 0) < bench.read_bytes(I, O, 2 * I * O, 0)
